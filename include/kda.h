@@ -1,0 +1,151 @@
+/*
+ * kda.h -- C ABI of the B200 (sm_100a) Kimi Delta Attention (KDA) library,
+ * libkda.so.
+ *
+ * The operator.  Per sequence n and head h, with a dk x dv fp32 state S
+ * (row = key channel, column = value channel):
+ *
+ *     S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T
+ *     o_t = S_t^T q_t,          alpha_t = exp(log_alpha_t)  (per key channel)
+ *
+ * Sources (page title and section):
+ *   - "Kimi Linear" summary (pt.news.hada.io), "Controle fino de memoria no
+ *     Kimi Delta Attention": a per-channel diagonal forget gate replaces the
+ *     scalar gate of Gated DeltaNet; the transition is a specialised
+ *     Diagonal-Plus-Low-Rank matrix tied to the key.
+ *   - same page, "Algoritmo paralelo por chunks": fixed-size chunks, the
+ *     final state of one chunk is the initial state of the next; WY / UT
+ *     representation; lower-triangular inverse by forward substitution;
+ *     output = inter-chunk recurrent term + intra-chunk parallel term.
+ *   - same page, "Da atencao linear ao Gated DeltaNet": the delta rule and its
+ *     Householder form.
+ *   The pages print no equation; the update above is the plainest reading of
+ *   their prose (decay first, output from the post-update state, no 1/sqrt(dk)
+ *   query scale, natural-log gates).
+ *
+ * Conventions for every entry point
+ * ---------------------------------
+ *   - All tensor arguments are DEVICE pointers owned by the caller; the
+ *     library never allocates, frees or retains them.  Calls are asynchronous
+ *     on `stream` (a cudaStream_t passed as void*; NULL = legacy default).
+ *   - Arguments are validated on the host before anything is launched; a
+ *     failing check returns an error status and launches nothing.
+ *   - The library never aborts, asserts, traps or prints.
+ *   - Pointers must be 16-byte aligned (KDA_ERR_ALIGN otherwise).
+ *   - Contiguous layouts (token-major, head next, channel innermost):
+ *       q, k, log_alpha : [B, T, H, dk]        v, o : [B, T, H, dv]
+ *       beta            : [B, T, H]
+ *       S0, S_T, S      : [N, H, dk, dv] fp32, dv innermost
+ *     With cu_seqlens (int32, N+1 non-decreasing offsets, cu[0] = 0,
+ *     cu[N] = T) the batch is packed: B must be 1, T is the packed total and
+ *     sequence n owns tokens [cu[n], cu[n+1]).  Without it N = B.
+ */
+#ifndef KDA_H_
+#define KDA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define KDA_ABI_VERSION 1
+
+typedef enum {
+  KDA_OK = 0,
+  KDA_ERR_NULL = -1,        /* a required pointer is NULL                     */
+  KDA_ERR_SHAPE = -2,       /* non-positive / inconsistent sizes              */
+  KDA_ERR_DTYPE = -3,       /* unknown dtype code                             */
+  KDA_ERR_ALIGN = -4,       /* a pointer is not 16-byte aligned               */
+  KDA_ERR_UNSUPPORTED = -5, /* valid but not implemented (e.g. dk not 64/128) */
+  KDA_ERR_WORKSPACE = -6,   /* workspace missing or smaller than required     */
+  KDA_ERR_CUDA = -7,        /* a CUDA runtime call or launch failed           */
+  KDA_ERR_TIMEOUT = -8,     /* a device-side bounded wait gave up             */
+  KDA_ERR_INTERNAL = -9,    /* a device-side consistency check failed         */
+  KDA_ERR_ARGUMENT = -10    /* other invalid argument (bad cu_seqlens, flags) */
+} kda_status;
+
+typedef enum { KDA_F32 = 0, KDA_BF16 = 1 } kda_dtype;
+
+/* Problem description shared by all entry points. */
+typedef struct kda_shape {
+  int32_t B;          /* batch rows (must be 1 when cu_seqlens is given)     */
+  int32_t T;          /* tokens per batch row; packed total with cu_seqlens  */
+  int32_t H;          /* heads                                               */
+  int32_t dk, dv;     /* key / value head dimensions: 64 or 128 each         */
+  int32_t chunk;      /* chunk length C of the chunkwise form: 16, 32 or 64  */
+  int32_t n_seqs;     /* N = number of packed sequences (with cu_seqlens)    */
+  int32_t io_dtype;   /* kda_dtype of q, k, v and o                          */
+  int32_t gate_dtype; /* kda_dtype of log_alpha and beta                     */
+  uint32_t flags;     /* KDA_FLAG_* bits                                     */
+} kda_shape;
+
+/* Copy cu_seqlens to the host and check it before launching.  This
+ * synchronises `stream`; without the flag cu_seqlens is trusted. */
+#define KDA_FLAG_VALIDATE_CU_SEQLENS 0x1u
+
+/*
+ * kda_chunk_fwd_workspace_size -- bytes of device workspace kda_chunk_fwd
+ * needs for `shape` (0 for paths that need none).  Returns 0 for shapes the
+ * library rejects; kda_chunk_fwd then reports the reason.
+ */
+size_t kda_chunk_fwd_workspace_size(const kda_shape* shape);
+
+/*
+ * kda_chunk_fwd -- chunkwise-parallel prefill ("Algoritmo paralelo por
+ * chunks" on the Kimi Linear summary page): runs the recurrence above over
+ * every token of every sequence and head, starting from S0.
+ *
+ *   q, k, log_alpha, v, beta  inputs (io_dtype / gate_dtype, layouts above).
+ *                             log_alpha <= 0 is expected (alpha in (0,1]).
+ *   S0          initial states [N, H, dk, dv] fp32, or NULL for zeros.
+ *   cu_seqlens  NULL for a dense batch, else N+1 int32 offsets (B == 1).
+ *   o           output [B, T, H, dv] in io_dtype; must not alias an input.
+ *   S_T         final states [N, H, dk, dv] fp32, or NULL; may alias S0.
+ *   workspace   device scratch of at least kda_chunk_fwd_workspace_size()
+ *               bytes (NULL allowed when that size is 0); contents on entry
+ *               are ignored and on exit undefined.
+ *
+ * Paths: bf16 io with dk = dv = 128 and chunk = 64 runs the tcgen05 tensor-
+ * core chunk kernels (fp32 state, bf16 operands, fp32 accumulation); every
+ * other supported shape, and all fp32 io, runs the fp32 CUDA-core recurrent
+ * kernel.  Sequences of length 0 copy S0 to S_T.
+ */
+kda_status kda_chunk_fwd(const kda_shape* shape, const void* q, const void* k, const void* v,
+                         const void* log_alpha, const void* beta, const float* S0,
+                         const int32_t* cu_seqlens, void* o, float* S_T, void* workspace,
+                         size_t workspace_bytes, void* stream);
+
+/*
+ * kda_decode_step -- one recurrent token for each of B independent
+ * (sequence, head) states, updated in place (the constant-size recurrent
+ * state of the "Kimi Linear" articles: one read and one write of S).
+ *
+ *   shape       B = number of sequences, T must be 1, chunk is ignored.
+ *   q, k, log_alpha : [B, H, dk];  v, o : [B, H, dv];  beta : [B, H].
+ *   S           [B, H, dk, dv] fp32, read and overwritten with the new state.
+ *   o           output; must not alias any input.
+ */
+kda_status kda_decode_step(const kda_shape* shape, const void* q, const void* k, const void* v,
+                           const void* log_alpha, const void* beta, float* S, void* o,
+                           void* stream);
+
+/*
+ * kda_check_device_error -- synchronises `stream`, then returns and clears
+ * the error code a kernel recorded on the current device (a bounded wait
+ * that gave up reports KDA_ERR_TIMEOUT).  KDA_OK when none was recorded.
+ */
+kda_status kda_check_device_error(void* stream);
+
+/* Static, human-readable text for a status code. */
+const char* kda_status_string(kda_status status);
+
+/* KDA_ABI_VERSION of the built library. */
+int32_t kda_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H_ */

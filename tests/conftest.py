@@ -1,0 +1,51 @@
+import os
+import sys
+from pathlib import Path
+
+import pytest
+
+ROOT = Path(__file__).resolve().parent.parent
+if str(ROOT) not in sys.path:
+    sys.path.insert(0, str(ROOT))
+
+
+def pytest_configure(config):
+    config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
+
+
+def pytest_collection_modifyitems(config, items):
+    # GPU tests are skipped (not failed) where no device exists, so the CPU
+    # suite can run with or without the marker filter.
+    try:
+        import torch
+        has_gpu = torch.cuda.is_available()
+    except Exception:  # pragma: no cover
+        has_gpu = False
+    if has_gpu:
+        return
+    skip = pytest.mark.skip(reason="no CUDA device")
+    for item in items:
+        if "gpu" in item.keywords:
+            item.add_marker(skip)
+
+
+def rel_l2(x, ref):
+    """max over leading slices of ||x - ref|| / max(||ref||, 1e-30)."""
+    import numpy as np
+    x = np.asarray(x, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    return float(np.linalg.norm(x - ref) / max(np.linalg.norm(ref), 1e-30))
+
+
+def max_rel_l2_per_slice(x, ref, slice_axes):
+    """Tolerance measure: the worst relative L2 error over (sequence, head) slices.
+
+    ``slice_axes`` are the axes that index slices; the others are reduced.
+    """
+    import numpy as np
+    x = np.asarray(x, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    other = tuple(a for a in range(x.ndim) if a not in slice_axes)
+    num = np.sqrt(((x - ref) ** 2).sum(axis=other))
+    den = np.maximum(np.sqrt((ref ** 2).sum(axis=other)), 1e-30)
+    return float((num / den).max())
