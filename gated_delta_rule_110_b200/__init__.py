@@ -1,0 +1,186 @@
+"""B200-native Kimi Delta Attention (KDA) operator.
+
+Python binding of ``libkda.so`` (the C ABI in ``include/kda.h``): argument
+marshalling only.  PyTorch supplies device memory and the current CUDA
+stream; every step of the operator runs in the library's sm_100a kernels.
+There is no CPU or PyTorch fallback: if the library cannot be loaded, or a
+tensor is not on a CUDA device, the call raises.
+
+Entry points (same names as the C ABI):
+
+* ``kda_chunk_fwd(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None)``
+  chunkwise-parallel prefill -> ``(o, S_T)``
+* ``kda_decode_step(q, k, v, log_alpha, beta, S)`` one recurrent token per
+  (sequence, head), ``S`` updated in place -> ``o``
+* ``kda_chunk_fwd_workspace_size(...)``, ``kda_check_device_error()``,
+  ``kda_status_string(code)``, ``kda_abi_version()``
+"""
+from __future__ import annotations
+
+import ctypes
+from pathlib import Path
+
+_PKG = Path(__file__).resolve().parent
+LIB_PATH = _PKG / "libkda.so"
+
+KDA_OK = 0
+KDA_F32, KDA_BF16 = 0, 1
+KDA_FLAG_VALIDATE_CU_SEQLENS = 0x1
+
+_STATUS_NAMES = {
+    0: "KDA_OK", -1: "KDA_ERR_NULL", -2: "KDA_ERR_SHAPE", -3: "KDA_ERR_DTYPE", -4: "KDA_ERR_ALIGN",
+    -5: "KDA_ERR_UNSUPPORTED", -6: "KDA_ERR_WORKSPACE", -7: "KDA_ERR_CUDA", -8: "KDA_ERR_TIMEOUT",
+    -9: "KDA_ERR_INTERNAL", -10: "KDA_ERR_ARGUMENT",
+}
+
+EXPORTED_SYMBOLS = (
+    "kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_decode_step", "kda_check_device_error",
+    "kda_status_string", "kda_abi_version",
+)
+
+
+class KdaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {_STATUS_NAMES.get(status, status)} ({kda_status_string(status)})")
+
+
+class kda_shape(ctypes.Structure):
+    _fields_ = [
+        ("B", ctypes.c_int32), ("T", ctypes.c_int32), ("H", ctypes.c_int32),
+        ("dk", ctypes.c_int32), ("dv", ctypes.c_int32), ("chunk", ctypes.c_int32),
+        ("n_seqs", ctypes.c_int32), ("io_dtype", ctypes.c_int32), ("gate_dtype", ctypes.c_int32),
+        ("flags", ctypes.c_uint32),
+    ]
+
+
+_lib = None
+
+
+def load_library(build_if_missing: bool = True):
+    """Load libkda.so (building it in-tree with nvcc if it is absent or stale)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if build_if_missing:
+        from . import build as _build
+        try:
+            _build.build()
+        except Exception as exc:  # no nvcc: only an existing library can be used
+            if not LIB_PATH.exists():
+                raise RuntimeError(f"libkda.so is missing and could not be built: {exc}") from exc
+    if not LIB_PATH.exists():
+        raise RuntimeError(f"libkda.so not found at {LIB_PATH}")
+    lib = ctypes.CDLL(str(LIB_PATH))
+    vp, sp = ctypes.c_void_p, ctypes.POINTER(kda_shape)
+    lib.kda_chunk_fwd_workspace_size.argtypes = [sp]
+    lib.kda_chunk_fwd_workspace_size.restype = ctypes.c_size_t
+    lib.kda_chunk_fwd.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
+    lib.kda_chunk_fwd.restype = ctypes.c_int
+    lib.kda_decode_step.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.kda_decode_step.restype = ctypes.c_int
+    lib.kda_check_device_error.argtypes = [vp]
+    lib.kda_check_device_error.restype = ctypes.c_int
+    lib.kda_status_string.argtypes = [ctypes.c_int]
+    lib.kda_status_string.restype = ctypes.c_char_p
+    lib.kda_abi_version.argtypes = []
+    lib.kda_abi_version.restype = ctypes.c_int32
+    _lib = lib
+    return lib
+
+
+def kda_status_string(status: int) -> str:
+    return load_library().kda_status_string(int(status)).decode()
+
+
+def kda_abi_version() -> int:
+    return int(load_library().kda_abi_version())
+
+
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.bfloat16:
+        return KDA_BF16
+    if t.dtype == torch.float32:
+        return KDA_F32
+    raise TypeError(f"unsupported dtype {t.dtype}: use torch.bfloat16 or torch.float32")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("all tensors must be CUDA tensors (the library has no CPU path)")
+        if t is not None and not t.is_contiguous():
+            raise ValueError("all tensors must be contiguous")
+
+
+def make_shape(B, T, H, dk, dv, chunk=64, n_seqs=0, io_dtype=KDA_BF16, gate_dtype=KDA_BF16, flags=0):
+    return kda_shape(B, T, H, dk, dv, chunk, n_seqs, io_dtype, gate_dtype, flags)
+
+
+def kda_chunk_fwd_workspace_size(shape: kda_shape) -> int:
+    return int(load_library().kda_chunk_fwd_workspace_size(ctypes.byref(shape)))
+
+
+def _shape_of(q, v, log_alpha, cu_seqlens, chunk, validate):
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    n_seqs = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
+    flags = KDA_FLAG_VALIDATE_CU_SEQLENS if validate else 0
+    return make_shape(B, T, H, dk, dv, chunk, n_seqs, _dtype_code(q), _dtype_code(log_alpha), flags)
+
+
+def kda_chunk_fwd(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, *, chunk: int = 64, o=None, S_T=None,
+                  workspace=None, stream=None, validate: bool = False, output_final_state: bool = True):
+    """Chunkwise KDA prefill.  Shapes as in include/kda.h; returns (o, S_T)."""
+    import torch
+    _need_cuda(q, k, v, log_alpha, beta, S0, cu_seqlens, o, S_T, workspace)
+    shape = _shape_of(q, v, log_alpha, cu_seqlens, chunk, validate)
+    N = shape.B if cu_seqlens is None else shape.n_seqs
+    if o is None:
+        o = torch.empty(v.shape, dtype=v.dtype, device=v.device)
+    if S_T is None and output_final_state:
+        S_T = torch.empty((N, shape.H, shape.dk, shape.dv), dtype=torch.float32, device=q.device)
+    need = kda_chunk_fwd_workspace_size(shape)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = load_library().kda_chunk_fwd(
+        ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0),
+        _ptr(cu_seqlens), _ptr(o), _ptr(S_T), _ptr(workspace), ws_bytes, _stream(stream))
+    if rc != KDA_OK:
+        raise KdaError(rc, "kda_chunk_fwd")
+    return o, S_T
+
+
+def kda_decode_step(q, k, v, log_alpha, beta, S, *, o=None, stream=None):
+    """One recurrent token: q, k, log_alpha [N,H,dk]; v [N,H,dv]; beta [N,H];
+    S [N,H,dk,dv] fp32 updated in place.  Returns o [N,H,dv]."""
+    import torch
+    _need_cuda(q, k, v, log_alpha, beta, S, o)
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    shape = make_shape(N, 1, H, dk, dv, 64, 0, _dtype_code(q), _dtype_code(log_alpha), 0)
+    if o is None:
+        o = torch.empty(v.shape, dtype=v.dtype, device=v.device)
+    rc = load_library().kda_decode_step(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
+                                        _ptr(beta), _ptr(S), _ptr(o), _stream(stream))
+    if rc != KDA_OK:
+        raise KdaError(rc, "kda_decode_step")
+    return o
+
+
+def kda_check_device_error(stream=None) -> int:
+    """Synchronise and return (and clear) the device-side error code."""
+    return int(load_library().kda_check_device_error(_stream(stream)))

@@ -1,0 +1,267 @@
+// kda_api.cu -- host side of libkda.so: argument validation, path selection
+// and kernel launches behind the extern "C" entry points of include/kda.h.
+// Every check runs on the host before anything is launched; no entry point
+// allocates device memory, aborts or prints.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <vector>
+
+#include "kda.h"
+#include "kda_chunk_tc.cuh"
+#include "kda_recurrent.cuh"
+
+namespace {
+
+using kda::tc::C;
+using kda::tc::SLOT_BYTES;
+
+inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+inline bool aligned16(const void* p) { return aligned(p, 16); }
+inline uintptr_t gate_size(const kda_shape& s) { return s.gate_dtype == KDA_BF16 ? 2 : 4; }
+// Alignment each kernel relies on: 16 bytes for fp32 states (float4) and the
+// workspace, 4 bytes for token tensors (bf16 pairs), element size for beta.
+inline bool token_ptrs_aligned(const kda_shape& s, const void* q, const void* k, const void* v, const void* la,
+                               const void* beta, const void* o) {
+  return aligned(q, 4) && aligned(k, 4) && aligned(v, 4) && aligned(la, 4) && aligned(o, 4) &&
+         aligned(beta, gate_size(s));
+}
+inline bool dtype_ok(int32_t d) { return d == KDA_F32 || d == KDA_BF16; }
+inline bool dim_ok(int32_t d) { return d == 64 || d == 128; }
+
+// Tensor-core chunk path: bf16 io, dk = dv = 128, C = 64.
+inline bool use_tc(const kda_shape& s) {
+  return s.io_dtype == KDA_BF16 && s.dk == 128 && s.dv == 128 && s.chunk == 64;
+}
+
+// Number of sequences N and the packed token total.
+inline void seq_counts(const kda_shape& s, const int32_t* cu, int64_t* N, int64_t* Ttot) {
+  if (cu) {
+    *N = s.n_seqs;
+    *Ttot = s.T;
+  } else {
+    *N = s.B;
+    *Ttot = static_cast<int64_t>(s.B) * s.T;
+  }
+}
+
+// Upper bound on the number of chunks over all sequences: each sequence of
+// length l has ceil(l / C) <= l / C + 1 chunks.
+inline int64_t max_chunks(int64_t N, int64_t Ttot) { return Ttot / C + N; }
+
+kda_status check_common(const kda_shape* sp) {
+  if (!sp) return KDA_ERR_NULL;
+  const kda_shape& s = *sp;
+  if (!dtype_ok(s.io_dtype) || !dtype_ok(s.gate_dtype)) return KDA_ERR_DTYPE;
+  if (s.B <= 0 || s.T < 0 || s.H <= 0) return KDA_ERR_SHAPE;
+  if (!dim_ok(s.dk) || !dim_ok(s.dv)) return KDA_ERR_UNSUPPORTED;
+  if ((s.flags & ~KDA_FLAG_VALIDATE_CU_SEQLENS) != 0u) return KDA_ERR_ARGUMENT;
+  return KDA_OK;
+}
+
+kda_status launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+template <int DK, int DV, typename TIO, typename TG>
+kda_status launch_recurrent_fwd(const kda_shape& s, int64_t N, const void* q, const void* k, const void* v,
+                                const void* la, const void* beta, const float* S0, const int32_t* cu, void* o,
+                                float* S_T, cudaStream_t st) {
+  dim3 grid(s.H, static_cast<unsigned>(N));
+  kda::kda_recurrent_fwd_kernel<DK, DV, TIO, TG><<<grid, kda::kRecThreads, 0, st>>>(
+      s.H, s.T, cu, static_cast<const TIO*>(q), static_cast<const TIO*>(k), static_cast<const TIO*>(v),
+      static_cast<const TG*>(la), static_cast<const TG*>(beta), S0, static_cast<TIO*>(o), S_T);
+  return launch_status();
+}
+
+template <typename TIO, typename TG>
+kda_status dispatch_recurrent_fwd(const kda_shape& s, int64_t N, const void* q, const void* k, const void* v,
+                                  const void* la, const void* beta, const float* S0, const int32_t* cu, void* o,
+                                  float* S_T, cudaStream_t st) {
+  if (s.dk == 128 && s.dv == 128)
+    return launch_recurrent_fwd<128, 128, TIO, TG>(s, N, q, k, v, la, beta, S0, cu, o, S_T, st);
+  if (s.dk == 64 && s.dv == 64)
+    return launch_recurrent_fwd<64, 64, TIO, TG>(s, N, q, k, v, la, beta, S0, cu, o, S_T, st);
+  if (s.dk == 128 && s.dv == 64)
+    return launch_recurrent_fwd<128, 64, TIO, TG>(s, N, q, k, v, la, beta, S0, cu, o, S_T, st);
+  return launch_recurrent_fwd<64, 128, TIO, TG>(s, N, q, k, v, la, beta, S0, cu, o, S_T, st);
+}
+
+template <int DK, int DV, typename TIO, typename TG>
+kda_status launch_decode(const kda_shape& s, const void* q, const void* k, const void* v, const void* la,
+                         const void* beta, float* S, void* o, cudaStream_t st) {
+  const unsigned blocks = static_cast<unsigned>(s.B) * static_cast<unsigned>(s.H);
+  kda::kda_decode_kernel<DK, DV, TIO, TG><<<blocks, kda::kRecThreads, 0, st>>>(
+      s.H, static_cast<const TIO*>(q), static_cast<const TIO*>(k), static_cast<const TIO*>(v),
+      static_cast<const TG*>(la), static_cast<const TG*>(beta), S, static_cast<TIO*>(o));
+  return launch_status();
+}
+
+template <typename TIO, typename TG>
+kda_status dispatch_decode(const kda_shape& s, const void* q, const void* k, const void* v, const void* la,
+                           const void* beta, float* S, void* o, cudaStream_t st) {
+  if (s.dk == 128 && s.dv == 128) return launch_decode<128, 128, TIO, TG>(s, q, k, v, la, beta, S, o, st);
+  if (s.dk == 64 && s.dv == 64) return launch_decode<64, 64, TIO, TG>(s, q, k, v, la, beta, S, o, st);
+  if (s.dk == 128 && s.dv == 64) return launch_decode<128, 64, TIO, TG>(s, q, k, v, la, beta, S, o, st);
+  return launch_decode<64, 128, TIO, TG>(s, q, k, v, la, beta, S, o, st);
+}
+
+// Per-device one-time opt-in to large dynamic shared memory.
+template <typename F>
+bool ensure_smem(F* kernel, uint32_t bytes, bool* done) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  if (done[dev]) return true;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes)) !=
+      cudaSuccess)
+    return false;
+  done[dev] = true;
+  return true;
+}
+
+template <typename TG>
+kda_status launch_tc(const kda_shape& s, int64_t N, int64_t Ttot, const void* q, const void* k, const void* v,
+                     const void* la, const void* beta, const float* S0, const int32_t* cu, void* o, float* S_T,
+                     void* ws, cudaStream_t st) {
+  static bool prep_ok[64] = {false}, rec_ok[64] = {false};
+  auto* prep = kda::tc::kda_chunk_prep_kernel<TG>;
+  auto* rec = kda::tc::kda_chunk_rec_kernel<__nv_bfloat16>;
+  if (!ensure_smem(prep, kda::tc::P_SMEM, prep_ok) || !ensure_smem(rec, kda::tc::R_SMEM, rec_ok))
+    return KDA_ERR_CUDA;
+  const int64_t mc = max_chunks(N, Ttot);
+  if (mc > 0) {
+    dim3 g1(static_cast<unsigned>(mc), static_cast<unsigned>(s.H));
+    prep<<<g1, 256, kda::tc::P_SMEM, st>>>(static_cast<int>(N), s.T, s.H, cu,
+                                           static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+                                           static_cast<const __nv_bfloat16*>(v), static_cast<const TG*>(la),
+                                           static_cast<const TG*>(beta), static_cast<uint8_t*>(ws));
+    const kda_status e = launch_status();
+    if (e != KDA_OK) return e;
+  }
+  dim3 g2(static_cast<unsigned>(s.H), static_cast<unsigned>(N));
+  rec<<<g2, kda::tc::REC_THREADS, kda::tc::R_SMEM, st>>>(static_cast<int>(N), s.T, s.H, cu,
+                                                         static_cast<const uint8_t*>(ws), S0,
+                                                         static_cast<__nv_bfloat16*>(o), S_T);
+  return launch_status();
+}
+
+kda_status validate_cu_host(const int32_t* cu, int64_t N, int64_t Ttot, cudaStream_t st) {
+  std::vector<int32_t> h(static_cast<size_t>(N) + 1);
+  if (cudaMemcpyAsync(h.data(), cu, h.size() * sizeof(int32_t), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return KDA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return KDA_ERR_CUDA;
+  if (h[0] != 0 || h[N] != Ttot) return KDA_ERR_ARGUMENT;
+  for (int64_t i = 0; i < N; ++i)
+    if (h[i + 1] < h[i]) return KDA_ERR_ARGUMENT;
+  return KDA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t kda_chunk_fwd_workspace_size(const kda_shape* sp) {
+  if (check_common(sp) != KDA_OK) return 0;
+  const kda_shape& s = *sp;
+  if (!use_tc(s)) return 0;
+  const bool packed = s.n_seqs > 0 && s.B == 1;
+  const int64_t N = packed ? s.n_seqs : s.B;
+  const int64_t Ttot = packed ? s.T : static_cast<int64_t>(s.B) * s.T;
+  return static_cast<size_t>(max_chunks(N, Ttot)) * static_cast<size_t>(s.H) * SLOT_BYTES;
+}
+
+kda_status kda_chunk_fwd(const kda_shape* sp, const void* q, const void* k, const void* v, const void* log_alpha,
+                         const void* beta, const float* S0, const int32_t* cu_seqlens, void* o, float* S_T,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+  kda_status e = check_common(sp);
+  if (e != KDA_OK) return e;
+  const kda_shape& s = *sp;
+  if (s.chunk != 16 && s.chunk != 32 && s.chunk != 64) return KDA_ERR_UNSUPPORTED;
+  if (cu_seqlens && (s.B != 1 || s.n_seqs <= 0)) return KDA_ERR_SHAPE;
+  int64_t N, Ttot;
+  seq_counts(s, cu_seqlens, &N, &Ttot);
+  const bool any_tokens = Ttot > 0;
+  if (any_tokens && (!q || !k || !v || !log_alpha || !beta || !o)) return KDA_ERR_NULL;
+  if (!token_ptrs_aligned(s, q, k, v, log_alpha, beta, o) || !aligned16(S0) || !aligned16(S_T) ||
+      !aligned(cu_seqlens, 4))
+    return KDA_ERR_ALIGN;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cu_seqlens && (s.flags & KDA_FLAG_VALIDATE_CU_SEQLENS)) {
+    e = validate_cu_host(cu_seqlens, N, Ttot, st);
+    if (e != KDA_OK) return e;
+  }
+  if (N == 0) return KDA_OK;
+
+  if (use_tc(s)) {
+    const size_t need = kda_chunk_fwd_workspace_size(sp);
+    if (need > 0 && (!workspace || workspace_bytes < need)) return KDA_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return KDA_ERR_ALIGN;
+    if (s.gate_dtype == KDA_BF16)
+      return launch_tc<__nv_bfloat16>(s, N, Ttot, q, k, v, log_alpha, beta, S0, cu_seqlens, o, S_T, workspace, st);
+    return launch_tc<float>(s, N, Ttot, q, k, v, log_alpha, beta, S0, cu_seqlens, o, S_T, workspace, st);
+  }
+  if (s.io_dtype == KDA_F32) {
+    if (s.gate_dtype == KDA_F32)
+      return dispatch_recurrent_fwd<float, float>(s, N, q, k, v, log_alpha, beta, S0, cu_seqlens, o, S_T, st);
+    return dispatch_recurrent_fwd<float, __nv_bfloat16>(s, N, q, k, v, log_alpha, beta, S0, cu_seqlens, o, S_T,
+                                                         st);
+  }
+  if (s.gate_dtype == KDA_F32)
+    return dispatch_recurrent_fwd<__nv_bfloat16, float>(s, N, q, k, v, log_alpha, beta, S0, cu_seqlens, o, S_T,
+                                                        st);
+  return dispatch_recurrent_fwd<__nv_bfloat16, __nv_bfloat16>(s, N, q, k, v, log_alpha, beta, S0, cu_seqlens, o,
+                                                              S_T, st);
+}
+
+kda_status kda_decode_step(const kda_shape* sp, const void* q, const void* k, const void* v, const void* log_alpha,
+                           const void* beta, float* S, void* o, void* stream) {
+  kda_status e = check_common(sp);
+  if (e != KDA_OK) return e;
+  const kda_shape& s = *sp;
+  if (s.T != 1) return KDA_ERR_SHAPE;
+  if (!q || !k || !v || !log_alpha || !beta || !S || !o) return KDA_ERR_NULL;
+  if (!token_ptrs_aligned(s, q, k, v, log_alpha, beta, o) || !aligned16(S)) return KDA_ERR_ALIGN;
+  if (static_cast<int64_t>(s.B) * s.H > 0x7fffffffLL) return KDA_ERR_SHAPE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (s.io_dtype == KDA_F32) {
+    if (s.gate_dtype == KDA_F32) return dispatch_decode<float, float>(s, q, k, v, log_alpha, beta, S, o, st);
+    return dispatch_decode<float, __nv_bfloat16>(s, q, k, v, log_alpha, beta, S, o, st);
+  }
+  if (s.gate_dtype == KDA_F32) return dispatch_decode<__nv_bfloat16, float>(s, q, k, v, log_alpha, beta, S, o, st);
+  return dispatch_decode<__nv_bfloat16, __nv_bfloat16>(s, q, k, v, log_alpha, beta, S, o, st);
+}
+
+kda_status kda_check_device_error(void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return KDA_ERR_CUDA;
+  int code = 0;
+  if (cudaMemcpyFromSymbol(&code, kda::g_device_error, sizeof(int)) != cudaSuccess) return KDA_ERR_CUDA;
+  if (code != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(kda::g_device_error, &zero, sizeof(int)) != cudaSuccess) return KDA_ERR_CUDA;
+  }
+  return static_cast<kda_status>(code);
+}
+
+const char* kda_status_string(kda_status status) {
+  switch (status) {
+    case KDA_OK: return "ok";
+    case KDA_ERR_NULL: return "a required pointer is NULL";
+    case KDA_ERR_SHAPE: return "invalid or inconsistent sizes";
+    case KDA_ERR_DTYPE: return "unknown dtype code";
+    case KDA_ERR_ALIGN: return "a pointer is not aligned as required";
+    case KDA_ERR_UNSUPPORTED: return "configuration not supported (dk, dv must be 64 or 128; chunk 16, 32 or 64)";
+    case KDA_ERR_WORKSPACE: return "workspace missing or too small";
+    case KDA_ERR_CUDA: return "a CUDA runtime call or kernel launch failed";
+    case KDA_ERR_TIMEOUT: return "a device-side bounded wait timed out";
+    case KDA_ERR_INTERNAL: return "a device-side consistency check failed";
+    case KDA_ERR_ARGUMENT: return "invalid argument (cu_seqlens or flags)";
+  }
+  return "unknown status";
+}
+
+int32_t kda_abi_version(void) { return KDA_ABI_VERSION; }
+
+}  // extern "C"

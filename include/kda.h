@@ -31,7 +31,9 @@
  *   - Arguments are validated on the host before anything is launched; a
  *     failing check returns an error status and launches nothing.
  *   - The library never aborts, asserts, traps or prints.
- *   - Pointers must be 16-byte aligned (KDA_ERR_ALIGN otherwise).
+ *   - Alignment (KDA_ERR_ALIGN otherwise): S0, S_T, S and the workspace
+ *     16 bytes; q, k, v, o and log_alpha 4 bytes; beta and cu_seqlens their
+ *     element size.
  *   - Contiguous layouts (token-major, head next, channel innermost):
  *       q, k, log_alpha : [B, T, H, dk]        v, o : [B, T, H, dv]
  *       beta            : [B, T, H]
@@ -57,7 +59,7 @@ typedef enum {
   KDA_ERR_NULL = -1,        /* a required pointer is NULL                     */
   KDA_ERR_SHAPE = -2,       /* non-positive / inconsistent sizes              */
   KDA_ERR_DTYPE = -3,       /* unknown dtype code                             */
-  KDA_ERR_ALIGN = -4,       /* a pointer is not 16-byte aligned               */
+  KDA_ERR_ALIGN = -4,       /* a pointer is not aligned as required           */
   KDA_ERR_UNSUPPORTED = -5, /* valid but not implemented (e.g. dk not 64/128) */
   KDA_ERR_WORKSPACE = -6,   /* workspace missing or smaller than required     */
   KDA_ERR_CUDA = -7,        /* a CUDA runtime call or launch failed           */

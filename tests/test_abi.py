@@ -1,0 +1,115 @@
+"""The C ABI boundary, checked on the host (no GPU needed).
+
+The library must load, export every entry point include/kda.h declares, and
+reject bad arguments with the documented status *before* launching anything.
+Only argument errors that are detected ahead of any CUDA call are exercised
+here, so no test ever hands a kernel a bogus pointer.
+"""
+import ctypes
+import re
+from pathlib import Path
+
+import pytest
+
+import gated_delta_rule_110_b200 as kda
+
+ROOT = Path(__file__).resolve().parents[1]
+
+
+def declared_functions():
+    text = (ROOT / "include" / "kda.h").read_text()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(kda_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_expected_entry_points():
+    assert declared_functions() == sorted(kda.EXPORTED_SYMBOLS)
+
+
+def test_library_loads_and_exports_every_declared_symbol():
+    lib = kda.load_library()
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert kda.kda_abi_version() == 1
+
+
+def test_status_strings():
+    for code in range(0, -11, -1):
+        s = kda.kda_status_string(code)
+        assert isinstance(s, str) and s and s != "unknown status"
+    assert kda.kda_status_string(-99) == "unknown status"
+
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: every call below fails validation first
+
+
+def call_fwd(shape, ptrs=None, ws=None, ws_bytes=0):
+    lib = kda.load_library()
+    p = dict(q=FAKE, k=FAKE, v=FAKE, la=FAKE, beta=FAKE, S0=None, cu=None, o=FAKE, ST=None)
+    p.update(ptrs or {})
+    vp = lambda x: None if x is None else ctypes.c_void_p(x)
+    return lib.kda_chunk_fwd(ctypes.byref(shape), vp(p["q"]), vp(p["k"]), vp(p["v"]), vp(p["la"]),
+                             vp(p["beta"]), vp(p["S0"]), vp(p["cu"]), vp(p["o"]), vp(p["ST"]), vp(ws), ws_bytes,
+                             None)
+
+
+def tc_shape(**kw):
+    base = dict(B=1, T=128, H=2, dk=128, dv=128, chunk=64, n_seqs=0, io_dtype=1, gate_dtype=1, flags=0)
+    base.update(kw)
+    return kda.make_shape(**base)
+
+
+def test_null_shape():
+    lib = kda.load_library()
+    assert lib.kda_chunk_fwd(None, *([None] * 9), None, 0, None) == -1
+    assert lib.kda_decode_step(None, *([None] * 7), None) == -1
+    assert lib.kda_chunk_fwd_workspace_size(None) == 0
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("io_dtype", 7, -3), ("gate_dtype", -1, -3), ("B", 0, -2), ("H", 0, -2), ("T", -1, -2),
+    ("dk", 96, -5), ("dv", 32, -5), ("chunk", 48, -5), ("flags", 0x80, -10),
+])
+def test_bad_shape_fields(field, value, status):
+    assert call_fwd(tc_shape(**{field: value})) == status
+
+
+def test_null_inputs_and_misalignment():
+    assert call_fwd(tc_shape(), {"q": None}) == -1
+    assert call_fwd(tc_shape(), {"o": None}) == -1
+    assert call_fwd(tc_shape(), {"k": FAKE + 2}) == -4
+    assert call_fwd(tc_shape(), {"beta": FAKE + 1}) == -4
+    assert call_fwd(tc_shape(), {"S0": FAKE + 8}) == -4
+
+
+def test_workspace_required_for_tensor_core_path():
+    s = tc_shape(B=2, T=200)
+    need = kda.kda_chunk_fwd_workspace_size(s)
+    # (floor(400/64) + 2 sequences) chunks x 2 heads x one 82,432-byte slot
+    assert need == (400 // 64 + 2) * 2 * 82432
+    assert call_fwd(s) == -6
+    assert call_fwd(s, ws=FAKE, ws_bytes=need - 16) == -6
+    assert call_fwd(s, ws=FAKE + 4, ws_bytes=need) == -4
+
+
+def test_cuda_core_path_needs_no_workspace():
+    assert kda.kda_chunk_fwd_workspace_size(tc_shape(io_dtype=0)) == 0
+    assert kda.kda_chunk_fwd_workspace_size(tc_shape(dk=64, dv=64)) == 0
+
+
+def test_packed_requires_single_batch_row():
+    assert call_fwd(tc_shape(B=2, n_seqs=3), {"cu": FAKE}) == -2
+
+
+def test_decode_rejects_multi_token():
+    lib = kda.load_library()
+    s = kda.make_shape(4, 2, 2, 128, 128)
+    args = [ctypes.c_void_p(FAKE)] * 7
+    assert lib.kda_decode_step(ctypes.byref(s), *args, None) == -2
+
+
+def test_python_binding_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros(1, 4, 1, 64)
+    with pytest.raises(ValueError):
+        kda.kda_chunk_fwd(x, x, x, x, torch.zeros(1, 4, 1))
