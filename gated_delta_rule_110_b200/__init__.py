@@ -34,8 +34,8 @@ _STATUS_NAMES = {
 }
 
 EXPORTED_SYMBOLS = (
-    "kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_decode_step", "kda_check_device_error",
-    "kda_status_string", "kda_abi_version",
+    "kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_chunk_fwd_noalloc", "kda_decode_step",
+    "kda_check_device_error", "kda_status_string", "kda_abi_version",
 )
 
 
@@ -77,6 +77,8 @@ def load_library(build_if_missing: bool = True):
     lib.kda_chunk_fwd_workspace_size.restype = ctypes.c_size_t
     lib.kda_chunk_fwd.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
     lib.kda_chunk_fwd.restype = ctypes.c_int
+    lib.kda_chunk_fwd_noalloc.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.kda_chunk_fwd_noalloc.restype = ctypes.c_int
     lib.kda_decode_step.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.kda_decode_step.restype = ctypes.c_int
     lib.kda_check_device_error.argtypes = [vp]
@@ -161,6 +163,23 @@ def kda_chunk_fwd(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, *, chunk: 
         _ptr(cu_seqlens), _ptr(o), _ptr(S_T), _ptr(workspace), ws_bytes, _stream(stream))
     if rc != KDA_OK:
         raise KdaError(rc, "kda_chunk_fwd")
+    return o, S_T
+
+
+def kda_chunk_fwd_noalloc(q, k, v, log_alpha, beta, S0, cu_seqlens, o, S_T, *, chunk: int = 64, stream=None):
+    """kda_chunk_fwd on the library's built-in scratch array (no workspace).
+
+    For callers that cannot allocate device memory where they run the prefill
+    (see include/kda.h for the size limit and the sharing rules).  o and S_T
+    are caller-owned outputs; nothing is allocated here.
+    """
+    _need_cuda(q, k, v, log_alpha, beta, S0, cu_seqlens, o, S_T)
+    shape = _shape_of(q, v, log_alpha, cu_seqlens, chunk, False)
+    rc = load_library().kda_chunk_fwd_noalloc(
+        ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0),
+        _ptr(cu_seqlens), _ptr(o), _ptr(S_T), _stream(stream))
+    if rc != KDA_OK:
+        raise KdaError(rc, "kda_chunk_fwd_noalloc")
     return o, S_T
 
 

@@ -6,6 +6,7 @@
 
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 #include <vector>
 
 #include "kda.h"
@@ -265,3 +266,51 @@ const char* kda_status_string(kda_status status) {
 int32_t kda_abi_version(void) { return KDA_ABI_VERSION; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// kda_chunk_fwd_noalloc: kda_chunk_fwd for callers that cannot allocate device
+// memory.  Its workspace is this file-scope array, reserved in the library's
+// device image on every GPU that loads the library and held until the process
+// exits.  Host code only ever sees a host-side stand-in for the array's name,
+// so the device address is looked up once per device with
+// cudaGetSymbolAddress, with that device current, and cached.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = static_cast<size_t>(KDA_NOALLOC_SCRATCH_BYTES);
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[64] = {};
+
+kda_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return KDA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return KDA_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return KDA_OK;
+}
+
+}  // namespace
+
+extern "C" kda_status kda_chunk_fwd_noalloc(const kda_shape* sp, const void* q, const void* k, const void* v,
+                                            const void* log_alpha, const void* beta, const float* S0,
+                                            const int32_t* cu_seqlens, void* o, float* S_T, void* stream) {
+  const kda_status e = check_common(sp);
+  if (e != KDA_OK) return e;
+  // the size check needs no CUDA call, so an oversized request launches nothing
+  const size_t need = kda_chunk_fwd_workspace_size(sp);
+  if (need > kNoAllocScratchBytes) return KDA_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  if (need > 0) {
+    const kda_status se = noalloc_scratch(&scratch);
+    if (se != KDA_OK) return se;
+  }
+  return kda_chunk_fwd(sp, q, k, v, log_alpha, beta, S0, cu_seqlens, o, S_T, scratch,
+                       need > 0 ? kNoAllocScratchBytes : 0, stream);
+}

@@ -120,6 +120,39 @@ kda_status kda_chunk_fwd(const kda_shape* shape, const void* q, const void* k, c
                          size_t workspace_bytes, void* stream);
 
 /*
+ * kda_chunk_fwd_noalloc -- kda_chunk_fwd for callers that cannot allocate.
+ *
+ * The pages have no counterpart to this call; it is a convenience of this
+ * library.  Some callers have no way to obtain device memory where they run
+ * the prefill: a plugin loaded into a framework whose memory pool already
+ * owns the GPU and offers no allocator across a C boundary, or a
+ * latency-critical serving loop that bans cudaMalloc because it synchronises
+ * the device and stalls every other stream.  This call takes the arguments of
+ * kda_chunk_fwd without the workspace and uses a fixed scratch array that
+ * lives in the library's device image instead.
+ *
+ *   - The array holds KDA_NOALLOC_SCRATCH_BYTES (64 MiB).  Every GPU that
+ *     loads the library reserves it until the process exits.
+ *   - A shape whose kda_chunk_fwd_workspace_size() exceeds that is rejected
+ *     with KDA_ERR_WORKSPACE before anything is launched (the tensor-core
+ *     path fits up to 814 (chunk, head) pairs, e.g. 16 heads x ~3,000 tokens;
+ *     shapes that need no workspace have no limit).
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture begins.
+ *   - Every call shares the one array, which keeps the last call's contents.
+ *     The kernels write every byte of it they later read, so nothing has to be
+ *     cleared between calls, but calls whose executions overlap on the GPU
+ *     (different streams or host threads) race on it: serialise them.
+ *   - It allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ */
+#define KDA_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+
+kda_status kda_chunk_fwd_noalloc(const kda_shape* shape, const void* q, const void* k, const void* v,
+                                 const void* log_alpha, const void* beta, const float* S0,
+                                 const int32_t* cu_seqlens, void* o, float* S_T, void* stream);
+
+/*
  * kda_decode_step -- one recurrent token for each of B independent
  * (sequence, head) states, updated in place (the constant-size recurrent
  * state of the "Kimi Linear" articles: one read and one write of S).

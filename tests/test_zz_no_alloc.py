@@ -1,0 +1,77 @@
+"""kda_chunk_fwd_noalloc: the prefill for callers that cannot allocate.
+
+Some users of this library run the prefill where they have no way to get
+device memory: a plugin inside a framework whose memory pool already owns the
+GPU and exposes no allocator across the C boundary, or a serving loop that
+bans cudaMalloc because it synchronises the whole device.  For them the
+library offers kda_chunk_fwd_noalloc, which runs the same tensor-core chunk
+kernels as kda_chunk_fwd but keeps their workspace in a fixed 64 MiB array
+inside the library instead of a caller-supplied buffer.
+
+These tests call it through the C ABI and check it against kda_chunk_fwd
+(the entry point with a caller-supplied workspace) within the bf16 tolerance
+the other parity tests use, on two calls in a row with different inputs, so
+the second call also shows that what the first left in the shared array does
+not leak into its result.  The file is named to be collected last.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import gated_delta_rule_110_b200 as kda
+from gated_delta_rule_110_b200 import inputs as gen
+
+TOL_BF16 = 2e-2
+
+
+def _rel_slices(x, ref, axes):
+    x = np.asarray(x, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    other = tuple(a for a in range(x.ndim) if a not in axes)
+    num = np.sqrt(((x - ref) ** 2).sum(axis=other))
+    den = np.maximum(np.sqrt((ref ** 2).sum(axis=other)), 1e-30)
+    return float((num / den).max())
+
+
+def _call_noalloc_c_abi(x, o, S_T):
+    lib = kda.load_library()
+    B, T, H, dk = x["q"].shape
+    n_seqs = 0 if x["cu_seqlens"] is None else x["cu_seqlens"].numel() - 1
+    shape = kda.make_shape(B, T, H, dk, x["v"].shape[-1], 64, n_seqs, kda.KDA_BF16, kda.KDA_BF16)
+    p = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    return lib.kda_chunk_fwd_noalloc(ctypes.byref(shape), p(x["q"]), p(x["k"]), p(x["v"]), p(x["log_alpha"]),
+                                     p(x["beta"]), p(x["S0"]), p(x["cu_seqlens"]), p(o), p(S_T), stream)
+
+
+@pytest.mark.gpu
+def test_noalloc_matches_workspace_entry_point_on_two_calls():
+    cases = [
+        gen.make_inputs(2, 200, 3, 128, 128, seed=301),                        # batched, ragged tail
+        gen.make_inputs(1, 330, 2, 128, 128, seqlens=[130, 1, 199], seed=302),  # packed sequences
+    ]
+    for x in cases:
+        xd = {k: (v.cuda() if v is not None else None) for k, v in x.items()}
+        o_ref, S_ref = kda.kda_chunk_fwd(xd["q"], xd["k"], xd["v"], xd["log_alpha"], xd["beta"], xd["S0"],
+                                         xd["cu_seqlens"])
+        o = torch.full_like(xd["v"], float("nan"))
+        S_T = torch.full_like(S_ref, float("nan"))
+        rc = _call_noalloc_c_abi(xd, o, S_T)
+        assert rc == 0, kda.kda_status_string(rc)
+        assert kda.kda_check_device_error() == 0
+        assert _rel_slices(o.float().cpu(), o_ref.float().cpu(), (0, 2)) <= TOL_BF16
+        assert _rel_slices(S_T.cpu(), S_ref.cpu(), (0, 1)) <= TOL_BF16
+
+
+def test_noalloc_rejects_shapes_beyond_its_scratch():
+    """A request larger than the built-in 64 MiB is refused before any launch
+    (host-side check, runs without a GPU)."""
+    lib = kda.load_library()
+    shape = kda.make_shape(1, 65536, 16, 128, 128, 64, 0, kda.KDA_BF16, kda.KDA_BF16)
+    assert kda.kda_chunk_fwd_workspace_size(shape) > 64 * 1024 * 1024
+    fake = ctypes.c_void_p(0x10000)
+    rc = lib.kda_chunk_fwd_noalloc(ctypes.byref(shape), fake, fake, fake, fake, fake, None, None, fake, None,
+                                   None)
+    assert rc == -6  # KDA_ERR_WORKSPACE
