@@ -29,10 +29,10 @@ used on the data path.
 from __future__ import annotations
 
 import argparse
+import faulthandler
 import json
 import os
 import statistics
-import subprocess
 import sys
 import threading
 import time
@@ -76,62 +76,84 @@ def decode_bytes(N, H, d, gate_bytes=2, io_bytes=2):
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason sampling during a timed region."""
+    """SM clock and throttle-reason sampling during a timed region.
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    Samples NVML every 5 ms on a background thread (dense enough for timed
+    regions of a few ms); without NVML the summary reports "unsampled".
+    """
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
-        self.lines = []
+    # NVML clocks-event-reason bits
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, cuda_index: int):
+        self.cuda_index = cuda_index
+        self.samples = []
+        self.max_mhz = None
+        self._stop = threading.Event()
         self._t = None
+        self._nvml = None
+        self._h = None
+
+    def _handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        self._nvml = pynvml
+        try:
+            # torch reports the PCI location as integers; NVML wants the
+            # "domain:bus:device.function" string as bytes
+            p = torch.cuda.get_device_properties(self.cuda_index)
+            bus = f"{int(p.pci_domain_id):08x}:{int(p.pci_bus_id):02x}:{int(p.pci_device_id):02x}.0".encode()
+            return pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            idx = self.cuda_index
+            if vis:
+                ids = [x.strip() for x in vis.split(",") if x.strip()]
+                if idx < len(ids) and ids[idx].isdigit():
+                    idx = int(ids[idx])
+            return pynvml.nvmlDeviceGetHandleByIndex(idx)
+
+    def _run(self):
+        nv = self._nvml
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons")
+        while not self._stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+                rs = get_reasons(self._h)
+                self.samples.append((sm, rs))
+            except Exception:
+                pass
+            time.sleep(0.005)
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self._t = threading.Thread(target=self._read, daemon=True)
+            self._h = self._handle()
+            self.max_mhz = self._nvml.nvmlDeviceGetMaxClockInfo(self._h, self._nvml.NVML_CLOCK_SM)
+            self._t = threading.Thread(target=self._run, daemon=True)
             self._t.start()
+            time.sleep(0.02)  # first samples before the timed region starts
         except Exception:
-            self.proc = None
+            self._t = None
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
-
     def __exit__(self, *a):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except Exception:
-                self.proc.kill()
-            if self._t is not None:
-                self._t.join(timeout=2)
+        self._stop.set()
+        if self._t is not None:
+            self._t.join(timeout=2)
 
     def summary(self):
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx.append(float(parts[2]))
-            except ValueError:
-                continue
-            for nm, val in zip(names, parts[5:9]):
-                if val.lower() == "active":
-                    reasons.add(nm)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unsampled"], "samples": 0,
+                    "source": "nvml"}
+        reasons = set()
+        for _, rs in self.samples:
+            for bit, name in self.REASONS.items():
+                if rs & bit:
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(x for x, _ in self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(self.samples), "source": "nvml"}
 
 
 def dist_setup():
@@ -262,8 +284,10 @@ def run_ours(args):
     def prefill():
         kda.kda_chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["S0"], o=o, S_T=S_T, workspace=ws)
 
+    progress("prefill: timing")
     with ClockSampler(local) as clk:
         t_pre = timed(prefill, args.steps, args.warmup, world, stream)
+    progress(f"prefill: {t_pre / args.steps * 1e3:.3f} ms/step")
     err = kda.kda_check_device_error()
     if err != 0:
         raise RuntimeError(f"device error {err} during prefill")
@@ -291,12 +315,14 @@ def run_ours(args):
         ho.copy_(o, non_blocking=True)
         hS.copy_(S_T, non_blocking=True)
 
+    progress("e2e: timing")
     e2e_steps = max(3, min(args.steps, 10))
     t_e2e = timed(e2e_step, e2e_steps, max(1, min(args.warmup, 3)), world, stream)
     e2e_value = tokens_per_step * world * e2e_steps / t_e2e
     del dx, hx
 
     # ---------------- decode
+    progress("decode: setup")
     wd = gen.workload("decode")
     Nd, Hd = wd.B, wd.H
     S = gen.decode_state(Nd, Hd, d, d, device="cuda", seed=wd.seed + rank)
@@ -320,8 +346,10 @@ def run_ours(args):
     dec_bytes = decode_bytes(Nd, Hd, d)
     dec_gbs = dec_bytes / (dec_ms / 1e3) / 1e9
 
+    progress(f"decode: {t_dec / dec_steps * 1e3:.3f} ms/step")
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        progress("cpu baseline")
         cpu = oracle_baseline(w)
 
     clocks = clk.summary()
@@ -335,7 +363,7 @@ def run_ours(args):
                        "B": B, "T": T, "H": H, "dk": d, "dv": d, "chunk": 64,
                        "l2": "inputs larger than L2 (no flush): 336 MB per step",
                        "parallelism": f"weak x{world}: each rank its own workload, no collective"},
-            "roofline": {"kernel": "kda_chunk_fwd (prep + recurrence launches)", "bound": "hbm",
+            "roofline": {"kernel": "kda_chunk_fused_kernel (one launch per call)", "bound": "hbm",
                          "achieved": achieved_gbs, "peak": peak_hbm, "unit": "GB/s",
                          "frac": achieved_gbs / peak_hbm, "traffic": None,
                          "algorithmic_bytes_per_launch": pre_bytes, "peak_source": peak_src,
@@ -344,7 +372,7 @@ def run_ours(args):
                                     "frac": pre_flops / (pre_ms / 1e3) / 1e12 / float(peaks["bf16_tflops"])}},
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": e2e_steps},
-            "gpu_launches": 2 * (args.steps + e2e_steps) + dec_steps,
+            "gpu_launches": (args.steps + e2e_steps) + dec_steps,
             "clocks": clocks,
             "decode": {"value": world * dec_steps / t_dec, "unit": "steps/s", "ms_per_step": dec_ms,
                        "steps": dec_steps,
@@ -365,7 +393,12 @@ def run_ours(args):
     return 0
 
 
+def progress(msg: str):
+    print(f"[bench] {msg}", file=sys.stderr, flush=True)
+
+
 def main():
+    faulthandler.enable()
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)

@@ -26,6 +26,7 @@ LIB_PATH = _PKG / "libkda.so"
 KDA_OK = 0
 KDA_F32, KDA_BF16 = 0, 1
 KDA_FLAG_VALIDATE_CU_SEQLENS = 0x1
+KDA_FLAG_PATH_TWO_PASS = 0x2
 
 _STATUS_NAMES = {
     0: "KDA_OK", -1: "KDA_ERR_NULL", -2: "KDA_ERR_SHAPE", -3: "KDA_ERR_DTYPE", -4: "KDA_ERR_ALIGN",
@@ -135,20 +136,24 @@ def kda_chunk_fwd_workspace_size(shape: kda_shape) -> int:
     return int(load_library().kda_chunk_fwd_workspace_size(ctypes.byref(shape)))
 
 
-def _shape_of(q, v, log_alpha, cu_seqlens, chunk, validate):
+def _shape_of(q, v, log_alpha, cu_seqlens, chunk, validate, two_pass=False):
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     n_seqs = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
-    flags = KDA_FLAG_VALIDATE_CU_SEQLENS if validate else 0
+    flags = (KDA_FLAG_VALIDATE_CU_SEQLENS if validate else 0) | (KDA_FLAG_PATH_TWO_PASS if two_pass else 0)
     return make_shape(B, T, H, dk, dv, chunk, n_seqs, _dtype_code(q), _dtype_code(log_alpha), flags)
 
 
 def kda_chunk_fwd(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, *, chunk: int = 64, o=None, S_T=None,
-                  workspace=None, stream=None, validate: bool = False, output_final_state: bool = True):
-    """Chunkwise KDA prefill.  Shapes as in include/kda.h; returns (o, S_T)."""
+                  workspace=None, stream=None, validate: bool = False, output_final_state: bool = True,
+                  two_pass: bool = False):
+    """Chunkwise KDA prefill.  Shapes as in include/kda.h; returns (o, S_T).
+
+    ``two_pass=True`` selects the prep + recurrence kernels (needs a workspace,
+    allocated here if not given) instead of the default fused kernel."""
     import torch
     _need_cuda(q, k, v, log_alpha, beta, S0, cu_seqlens, o, S_T, workspace)
-    shape = _shape_of(q, v, log_alpha, cu_seqlens, chunk, validate)
+    shape = _shape_of(q, v, log_alpha, cu_seqlens, chunk, validate, two_pass)
     N = shape.B if cu_seqlens is None else shape.n_seqs
     if o is None:
         o = torch.empty(v.shape, dtype=v.dtype, device=v.device)

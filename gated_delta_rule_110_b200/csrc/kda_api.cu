@@ -10,6 +10,7 @@
 #include <vector>
 
 #include "kda.h"
+#include "kda_chunk_fused.cuh"
 #include "kda_chunk_tc.cuh"
 #include "kda_recurrent.cuh"
 
@@ -31,10 +32,14 @@ inline bool token_ptrs_aligned(const kda_shape& s, const void* q, const void* k,
 inline bool dtype_ok(int32_t d) { return d == KDA_F32 || d == KDA_BF16; }
 inline bool dim_ok(int32_t d) { return d == 64 || d == 128; }
 
-// Tensor-core chunk path: bf16 io, dk = dv = 128, C = 64.
+// Tensor-core chunk path: bf16 io, dk = dv = 128, C = 64.  It runs the fused
+// single-kernel form unless KDA_FLAG_PATH_TWO_PASS asks for the two-kernel
+// form (prep + recurrence through a workspace).
 inline bool use_tc(const kda_shape& s) {
   return s.io_dtype == KDA_BF16 && s.dk == 128 && s.dv == 128 && s.chunk == 64;
 }
+inline bool use_two_pass(const kda_shape& s) { return use_tc(s) && (s.flags & KDA_FLAG_PATH_TWO_PASS) != 0u; }
+constexpr uint32_t kKnownFlags = KDA_FLAG_VALIDATE_CU_SEQLENS | KDA_FLAG_PATH_TWO_PASS;
 
 // Number of sequences N and the packed token total.
 inline void seq_counts(const kda_shape& s, const int32_t* cu, int64_t* N, int64_t* Ttot) {
@@ -57,7 +62,7 @@ kda_status check_common(const kda_shape* sp) {
   if (!dtype_ok(s.io_dtype) || !dtype_ok(s.gate_dtype)) return KDA_ERR_DTYPE;
   if (s.B <= 0 || s.T < 0 || s.H <= 0) return KDA_ERR_SHAPE;
   if (!dim_ok(s.dk) || !dim_ok(s.dv)) return KDA_ERR_UNSUPPORTED;
-  if ((s.flags & ~KDA_FLAG_VALIDATE_CU_SEQLENS) != 0u) return KDA_ERR_ARGUMENT;
+  if ((s.flags & ~kKnownFlags) != 0u) return KDA_ERR_ARGUMENT;
   return KDA_OK;
 }
 
@@ -148,6 +153,20 @@ kda_status launch_tc(const kda_shape& s, int64_t N, int64_t Ttot, const void* q,
   return launch_status();
 }
 
+template <typename TG>
+kda_status launch_fused(const kda_shape& s, int64_t N, const void* q, const void* k, const void* v, const void* la,
+                        const void* beta, const float* S0, const int32_t* cu, void* o, float* S_T, cudaStream_t st) {
+  static bool ok[64] = {false};
+  auto* kern = kda::fused::kda_chunk_fused_kernel<TG>;
+  if (!ensure_smem(kern, kda::fused::SMEM_BYTES, ok)) return KDA_ERR_CUDA;
+  dim3 grid(static_cast<unsigned>(s.H), static_cast<unsigned>(N));
+  kern<<<grid, kda::fused::NTHREADS, kda::fused::SMEM_BYTES, st>>>(
+      s.T, s.H, cu, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+      static_cast<const __nv_bfloat16*>(v), static_cast<const TG*>(la), static_cast<const TG*>(beta), S0,
+      static_cast<__nv_bfloat16*>(o), S_T);
+  return launch_status();
+}
+
 kda_status validate_cu_host(const int32_t* cu, int64_t N, int64_t Ttot, cudaStream_t st) {
   std::vector<int32_t> h(static_cast<size_t>(N) + 1);
   if (cudaMemcpyAsync(h.data(), cu, h.size() * sizeof(int32_t), cudaMemcpyDeviceToHost, st) != cudaSuccess)
@@ -166,7 +185,7 @@ extern "C" {
 size_t kda_chunk_fwd_workspace_size(const kda_shape* sp) {
   if (check_common(sp) != KDA_OK) return 0;
   const kda_shape& s = *sp;
-  if (!use_tc(s)) return 0;
+  if (!use_two_pass(s)) return 0;
   const bool packed = s.n_seqs > 0 && s.B == 1;
   const int64_t N = packed ? s.n_seqs : s.B;
   const int64_t Ttot = packed ? s.T : static_cast<int64_t>(s.B) * s.T;
@@ -195,7 +214,12 @@ kda_status kda_chunk_fwd(const kda_shape* sp, const void* q, const void* k, cons
   }
   if (N == 0) return KDA_OK;
 
-  if (use_tc(s)) {
+  if (use_tc(s) && !use_two_pass(s)) {
+    if (s.gate_dtype == KDA_BF16)
+      return launch_fused<__nv_bfloat16>(s, N, q, k, v, log_alpha, beta, S0, cu_seqlens, o, S_T, st);
+    return launch_fused<float>(s, N, q, k, v, log_alpha, beta, S0, cu_seqlens, o, S_T, st);
+  }
+  if (use_two_pass(s)) {
     const size_t need = kda_chunk_fwd_workspace_size(sp);
     if (need > 0 && (!workspace || workspace_bytes < need)) return KDA_ERR_WORKSPACE;
     if (!aligned16(workspace)) return KDA_ERR_ALIGN;
@@ -298,11 +322,15 @@ kda_status noalloc_scratch(void** out) {
 
 }  // namespace
 
-extern "C" kda_status kda_chunk_fwd_noalloc(const kda_shape* sp, const void* q, const void* k, const void* v,
+extern "C" kda_status kda_chunk_fwd_noalloc(const kda_shape* sp_in, const void* q, const void* k, const void* v,
                                             const void* log_alpha, const void* beta, const float* S0,
                                             const int32_t* cu_seqlens, void* o, float* S_T, void* stream) {
-  const kda_status e = check_common(sp);
+  const kda_status e = check_common(sp_in);
   if (e != KDA_OK) return e;
+  // the two-pass kernels are the ones that need scratch; run them on the array
+  kda_shape shape = *sp_in;
+  shape.flags |= KDA_FLAG_PATH_TWO_PASS;
+  const kda_shape* sp = &shape;
   // the size check needs no CUDA call, so an oversized request launches nothing
   const size_t need = kda_chunk_fwd_workspace_size(sp);
   if (need > kNoAllocScratchBytes) return KDA_ERR_WORKSPACE;

@@ -286,7 +286,7 @@ __global__ void __launch_bounds__(256, 1)
       mma_commit(bar_ap);
     }
     if (warp < 4) {
-      mbar_wait(bar_ap, 0, abort_flag);
+      mbar_wait_warp(bar_ap, 0, abort_flag);
       tc_fence_after();
       float x0[32], x1[32];
       const uint32_t ta = tmem + (static_cast<uint32_t>(32 * warp) << 16);
@@ -436,7 +436,7 @@ __global__ void __launch_bounds__(256, 1)
     mma_commit(bar_w);
   }
   if (warp < 4) {
-    mbar_wait(bar_w, 0, abort_flag);
+    mbar_wait_warp(bar_w, 0, abort_flag);
     tc_fence_after();
     // M = 64 accumulator: row 16w + i lives in TMEM lane 32w + i (i < 16)
     const uint32_t ta = tmem + (static_cast<uint32_t>(32 * warp) << 16) + 64;
@@ -660,7 +660,7 @@ __global__ void __launch_bounds__(REC_THREADS, 1)
       const uint32_t d1 = lane_base + tm_d1(b);
 
       // U^T -> bf16 operand
-      if (!mbar_wait(d1_full, j & 1, abort_flag)) break;
+      if (!mbar_wait_warp(d1_full, j & 1, abort_flag)) break;
       tc_fence_after();
       {
         float x[32];
@@ -681,7 +681,7 @@ __global__ void __launch_bounds__(REC_THREADS, 1)
       mbar_arrive(u_ready);
 
       // S <- gamma_C S + dS ; bf16 S^T for the next chunk
-      if (!mbar_wait(d2_full, j & 1, abort_flag)) break;
+      if (!mbar_wait_warp(d2_full, j & 1, abort_flag)) break;
       tc_fence_after();
       {
         const float* gC = reinterpret_cast<const float*>(slotp + GC_OFF) + 64 * hf;

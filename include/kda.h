@@ -86,11 +86,17 @@ typedef struct kda_shape {
 /* Copy cu_seqlens to the host and check it before launching.  This
  * synchronises `stream`; without the flag cu_seqlens is trusted. */
 #define KDA_FLAG_VALIDATE_CU_SEQLENS 0x1u
+/* Run the tensor-core chunk path as two kernels (a fully parallel prep over
+ * every (chunk, head) writing MMA-ready operands to the workspace, then the
+ * inter-chunk recurrence) instead of the default single fused kernel. */
+#define KDA_FLAG_PATH_TWO_PASS 0x2u
 
 /*
  * kda_chunk_fwd_workspace_size -- bytes of device workspace kda_chunk_fwd
- * needs for `shape` (0 for paths that need none).  Returns 0 for shapes the
- * library rejects; kda_chunk_fwd then reports the reason.
+ * needs for `shape`: 0 except on the two-pass tensor-core path
+ * (KDA_FLAG_PATH_TWO_PASS), which needs one 82,432-byte operand slot per
+ * (chunk, head).  Returns 0 for shapes the library rejects; kda_chunk_fwd
+ * then reports the reason.
  */
 size_t kda_chunk_fwd_workspace_size(const kda_shape* shape);
 
@@ -109,10 +115,12 @@ size_t kda_chunk_fwd_workspace_size(const kda_shape* shape);
  *               bytes (NULL allowed when that size is 0); contents on entry
  *               are ignored and on exit undefined.
  *
- * Paths: bf16 io with dk = dv = 128 and chunk = 64 runs the tcgen05 tensor-
- * core chunk kernels (fp32 state, bf16 operands, fp32 accumulation); every
- * other supported shape, and all fp32 io, runs the fp32 CUDA-core recurrent
- * kernel.  Sequences of length 0 copy S0 to S_T.
+ * Paths: bf16 io with dk = dv = 128 and chunk = 64 runs on the tcgen05
+ * tensor cores (fp32 state, bf16 operands, fp32 accumulation): by default one
+ * fused kernel per call, one CTA per (sequence, head), no workspace; with
+ * KDA_FLAG_PATH_TWO_PASS a prep kernel plus a recurrence kernel through the
+ * workspace.  Every other supported shape, and all fp32 io, runs the fp32
+ * CUDA-core recurrent kernel.  Sequences of length 0 copy S0 to S_T.
  */
 kda_status kda_chunk_fwd(const kda_shape* shape, const void* q, const void* k, const void* v,
                          const void* log_alpha, const void* beta, const float* S0,
@@ -128,8 +136,10 @@ kda_status kda_chunk_fwd(const kda_shape* shape, const void* q, const void* k, c
  * owns the GPU and offers no allocator across a C boundary, or a
  * latency-critical serving loop that bans cudaMalloc because it synchronises
  * the device and stalls every other stream.  This call takes the arguments of
- * kda_chunk_fwd without the workspace and uses a fixed scratch array that
- * lives in the library's device image instead.
+ * kda_chunk_fwd without the workspace and runs the two-pass tensor-core path
+ * (the one that needs scratch, KDA_FLAG_PATH_TWO_PASS) on a fixed scratch
+ * array that lives in the library's device image.  (The default fused path of
+ * kda_chunk_fwd needs no workspace at all.)
  *
  *   - The array holds KDA_NOALLOC_SCRATCH_BYTES (64 MiB).  Every GPU that
  *     loads the library reserves it until the process exits.

@@ -82,8 +82,8 @@ def test_null_inputs_and_misalignment():
     assert call_fwd(tc_shape(), {"S0": FAKE + 8}) == -4
 
 
-def test_workspace_required_for_tensor_core_path():
-    s = tc_shape(B=2, T=200)
+def test_workspace_required_for_two_pass_path():
+    s = tc_shape(B=2, T=200, flags=kda.KDA_FLAG_PATH_TWO_PASS)
     need = kda.kda_chunk_fwd_workspace_size(s)
     # (floor(400/64) + 2 sequences) chunks x 2 heads x one 82,432-byte slot
     assert need == (400 // 64 + 2) * 2 * 82432
@@ -92,7 +92,8 @@ def test_workspace_required_for_tensor_core_path():
     assert call_fwd(s, ws=FAKE + 4, ws_bytes=need) == -4
 
 
-def test_cuda_core_path_needs_no_workspace():
+def test_fused_and_cuda_core_paths_need_no_workspace():
+    assert kda.kda_chunk_fwd_workspace_size(tc_shape()) == 0
     assert kda.kda_chunk_fwd_workspace_size(tc_shape(io_dtype=0)) == 0
     assert kda.kda_chunk_fwd_workspace_size(tc_shape(dk=64, dv=64)) == 0
 

@@ -4,15 +4,15 @@ Some users of this library run the prefill where they have no way to get
 device memory: a plugin inside a framework whose memory pool already owns the
 GPU and exposes no allocator across the C boundary, or a serving loop that
 bans cudaMalloc because it synchronises the whole device.  For them the
-library offers kda_chunk_fwd_noalloc, which runs the same tensor-core chunk
-kernels as kda_chunk_fwd but keeps their workspace in a fixed 64 MiB array
-inside the library instead of a caller-supplied buffer.
+library offers kda_chunk_fwd_noalloc, which runs the two-pass tensor-core
+chunk kernels (the path that needs scratch) with their workspace in a fixed
+64 MiB array inside the library instead of a caller-supplied buffer.
 
 These tests call it through the C ABI and check it against kda_chunk_fwd
-(the entry point with a caller-supplied workspace) within the bf16 tolerance
-the other parity tests use, on two calls in a row with different inputs, so
-the second call also shows that what the first left in the shared array does
-not leak into its result.  The file is named to be collected last.
+within the bf16 tolerance the other parity tests use, on two calls in a row
+with different inputs, so the second call also shows that what the first left
+in the shared array does not leak into its result.  The file is named to be
+collected last.
 """
 import ctypes
 
@@ -70,7 +70,9 @@ def test_noalloc_rejects_shapes_beyond_its_scratch():
     (host-side check, runs without a GPU)."""
     lib = kda.load_library()
     shape = kda.make_shape(1, 65536, 16, 128, 128, 64, 0, kda.KDA_BF16, kda.KDA_BF16)
-    assert kda.kda_chunk_fwd_workspace_size(shape) > 64 * 1024 * 1024
+    two_pass = kda.make_shape(1, 65536, 16, 128, 128, 64, 0, kda.KDA_BF16, kda.KDA_BF16,
+                              kda.KDA_FLAG_PATH_TWO_PASS)
+    assert kda.kda_chunk_fwd_workspace_size(two_pass) > 64 * 1024 * 1024
     fake = ctypes.c_void_p(0x10000)
     rc = lib.kda_chunk_fwd_noalloc(ctypes.byref(shape), fake, fake, fake, fake, fake, None, None, fake, None,
                                    None)
