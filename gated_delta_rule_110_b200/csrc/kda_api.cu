@@ -6,7 +6,6 @@
 
 #include <cstdint>
 #include <cstring>
-#include <mutex>
 #include <vector>
 
 #include "kda.h"
@@ -114,28 +113,22 @@ kda_status dispatch_decode(const kda_shape& s, const void* q, const void* k, con
   return launch_decode<64, 128, TIO, TG>(s, q, k, v, la, beta, S, o, st);
 }
 
-// Per-device one-time opt-in to large dynamic shared memory.
+// Opt-in to large dynamic shared memory.  Set on every launch: the call is
+// a cheap host-side attribute update, and caching it per device would go
+// stale if the caller resets the device (the attribute dies with the context).
 template <typename F>
-bool ensure_smem(F* kernel, uint32_t bytes, bool* done) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
-  if (done[dev]) return true;
-  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes)) !=
-      cudaSuccess)
-    return false;
-  done[dev] = true;
-  return true;
+bool ensure_smem(F* kernel, uint32_t bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes)) ==
+         cudaSuccess;
 }
 
 template <typename TG>
 kda_status launch_tc(const kda_shape& s, int64_t N, int64_t Ttot, const void* q, const void* k, const void* v,
                      const void* la, const void* beta, const float* S0, const int32_t* cu, void* o, float* S_T,
                      void* ws, cudaStream_t st) {
-  static bool prep_ok[64] = {false}, rec_ok[64] = {false};
   auto* prep = kda::tc::kda_chunk_prep_kernel<TG>;
   auto* rec = kda::tc::kda_chunk_rec_kernel<__nv_bfloat16>;
-  if (!ensure_smem(prep, kda::tc::P_SMEM, prep_ok) || !ensure_smem(rec, kda::tc::R_SMEM, rec_ok))
-    return KDA_ERR_CUDA;
+  if (!ensure_smem(prep, kda::tc::P_SMEM) || !ensure_smem(rec, kda::tc::R_SMEM)) return KDA_ERR_CUDA;
   const int64_t mc = max_chunks(N, Ttot);
   if (mc > 0) {
     dim3 g1(static_cast<unsigned>(mc), static_cast<unsigned>(s.H));
@@ -156,9 +149,8 @@ kda_status launch_tc(const kda_shape& s, int64_t N, int64_t Ttot, const void* q,
 template <typename TG>
 kda_status launch_fused(const kda_shape& s, int64_t N, const void* q, const void* k, const void* v, const void* la,
                         const void* beta, const float* S0, const int32_t* cu, void* o, float* S_T, cudaStream_t st) {
-  static bool ok[64] = {false};
   auto* kern = kda::fused::kda_chunk_fused_kernel<TG>;
-  if (!ensure_smem(kern, kda::fused::SMEM_BYTES, ok)) return KDA_ERR_CUDA;
+  if (!ensure_smem(kern, kda::fused::SMEM_BYTES)) return KDA_ERR_CUDA;
   dim3 grid(static_cast<unsigned>(s.H), static_cast<unsigned>(N));
   kern<<<grid, kda::fused::NTHREADS, kda::fused::SMEM_BYTES, st>>>(
       s.T, s.H, cu, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
@@ -296,27 +288,21 @@ int32_t kda_abi_version(void) { return KDA_ABI_VERSION; }
 // memory.  Its workspace is this file-scope array, reserved in the library's
 // device image on every GPU that loads the library and held until the process
 // exits.  Host code only ever sees a host-side stand-in for the array's name,
-// so the device address is looked up once per device with
-// cudaGetSymbolAddress, with that device current, and cached.
+// so the device address is looked up with cudaGetSymbolAddress, with the
+// caller's device current, on every call.  The lookup allocates nothing and
+// costs a host-side table read once the module is loaded; not caching it
+// means a device reset (which reloads the module at a new address) can never
+// leave a stale pointer behind.
 // ---------------------------------------------------------------------------
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = static_cast<size_t>(KDA_NOALLOC_SCRATCH_BYTES);
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
-std::mutex g_noalloc_mutex;
-void* g_noalloc_ptr[64] = {};
-
 kda_status noalloc_scratch(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return KDA_ERR_CUDA;
-  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-  if (!g_noalloc_ptr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return KDA_ERR_CUDA;
-    g_noalloc_ptr[dev] = p;
-  }
-  *out = g_noalloc_ptr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return KDA_ERR_CUDA;
+  *out = p;
   return KDA_OK;
 }
 

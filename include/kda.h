@@ -147,9 +147,10 @@ kda_status kda_chunk_fwd(const kda_shape* shape, const void* q, const void* k, c
  *     with KDA_ERR_WORKSPACE before anything is launched (the tensor-core
  *     path fits up to 814 (chunk, head) pairs, e.g. 16 heads x ~3,000 tokens;
  *     shapes that need no workspace have no limit).
- *   - The first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture begins.
+ *   - Every call looks up the array's device address (cudaGetSymbolAddress)
+ *     on the current device; the lookup allocates nothing.  The first call on
+ *     a device may load the library's device code there, so make that first
+ *     call before any stream capture begins.
  *   - Every call shares the one array, which keeps the last call's contents.
  *     The kernels write every byte of it they later read, so nothing has to be
  *     cleared between calls, but calls whose executions overlap on the GPU

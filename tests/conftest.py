@@ -30,7 +30,7 @@ def pytest_collection_modifyitems(config, items):
 
 
 def rel_l2(x, ref):
-    """max over leading slices of ||x - ref|| / max(||ref||, 1e-30)."""
+    """||x - ref|| / max(||ref||, 1e-30) over the whole array."""
     import numpy as np
     x = np.asarray(x, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
@@ -49,3 +49,24 @@ def max_rel_l2_per_slice(x, ref, slice_axes):
     num = np.sqrt(((x - ref) ** 2).sum(axis=other))
     den = np.maximum(np.sqrt((ref ** 2).sum(axis=other)), 1e-30)
     return float((num / den).max())
+
+
+def max_rel_l2_per_window(x, ref, window=64):
+    """Worst relative L2 error over token windows of one sequence.
+
+    ``x`` and ``ref`` are [tokens, heads, dv] for ONE sequence, tokens counted
+    from the sequence start.  Each (window, head) block of ``window`` tokens
+    (the last one ragged) is compared on its own, so an error confined to one
+    chunk is not diluted by the rest of a long sequence.
+    """
+    import numpy as np
+    x = np.asarray(x, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    T = x.shape[0]
+    worst = 0.0
+    for a in range(0, T, window):
+        d = x[a:a + window] - ref[a:a + window]
+        num = np.sqrt((d ** 2).sum(axis=(0, 2)))
+        den = np.maximum(np.sqrt((ref[a:a + window] ** 2).sum(axis=(0, 2))), 1e-30)
+        worst = max(worst, float((num / den).max()))
+    return worst
