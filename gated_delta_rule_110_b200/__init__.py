@@ -136,24 +136,35 @@ def kda_chunk_fwd_workspace_size(shape: kda_shape) -> int:
     return int(load_library().kda_chunk_fwd_workspace_size(ctypes.byref(shape)))
 
 
-def _shape_of(q, v, log_alpha, cu_seqlens, chunk, validate, two_pass=False):
+def tuning_flags(state_ctas: int = 0, grid_ctas: int = 0) -> int:
+    """Flag bits fixing the number of state CTAs / capping the grid of the
+    pipelined tensor-core path (0 = automatic), as in include/kda.h."""
+    if not (0 <= state_ctas <= 255 and 0 <= grid_ctas <= 255):
+        raise ValueError("state_ctas and grid_ctas must be in [0, 255]")
+    return (state_ctas << 8) | (grid_ctas << 16)
+
+
+def _shape_of(q, v, log_alpha, cu_seqlens, chunk, validate, two_pass=False, state_ctas=0, grid_ctas=0):
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     n_seqs = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
     flags = (KDA_FLAG_VALIDATE_CU_SEQLENS if validate else 0) | (KDA_FLAG_PATH_TWO_PASS if two_pass else 0)
+    flags |= tuning_flags(state_ctas, grid_ctas)
     return make_shape(B, T, H, dk, dv, chunk, n_seqs, _dtype_code(q), _dtype_code(log_alpha), flags)
 
 
 def kda_chunk_fwd(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, *, chunk: int = 64, o=None, S_T=None,
                   workspace=None, stream=None, validate: bool = False, output_final_state: bool = True,
-                  two_pass: bool = False):
+                  two_pass: bool = False, state_ctas: int = 0, grid_ctas: int = 0):
     """Chunkwise KDA prefill.  Shapes as in include/kda.h; returns (o, S_T).
 
-    ``two_pass=True`` selects the prep + recurrence kernels (needs a workspace,
-    allocated here if not given) instead of the default fused kernel."""
+    The tensor-core path needs a workspace (allocated here from PyTorch's
+    caching allocator if not given).  ``two_pass=True`` selects the prep +
+    recurrence kernels instead of the default pipelined kernel;
+    ``state_ctas`` / ``grid_ctas`` override its CTA split (0 = automatic)."""
     import torch
     _need_cuda(q, k, v, log_alpha, beta, S0, cu_seqlens, o, S_T, workspace)
-    shape = _shape_of(q, v, log_alpha, cu_seqlens, chunk, validate, two_pass)
+    shape = _shape_of(q, v, log_alpha, cu_seqlens, chunk, validate, two_pass, state_ctas, grid_ctas)
     N = shape.B if cu_seqlens is None else shape.n_seqs
     if o is None:
         o = torch.empty(v.shape, dtype=v.dtype, device=v.device)
@@ -171,7 +182,8 @@ def kda_chunk_fwd(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, *, chunk: 
     return o, S_T
 
 
-def kda_chunk_fwd_noalloc(q, k, v, log_alpha, beta, S0, cu_seqlens, o, S_T, *, chunk: int = 64, stream=None):
+def kda_chunk_fwd_noalloc(q, k, v, log_alpha, beta, S0, cu_seqlens, o, S_T, *, chunk: int = 64, stream=None,
+                          two_pass: bool = False):
     """kda_chunk_fwd on the library's built-in scratch array (no workspace).
 
     For callers that cannot allocate device memory where they run the prefill
@@ -179,7 +191,7 @@ def kda_chunk_fwd_noalloc(q, k, v, log_alpha, beta, S0, cu_seqlens, o, S_T, *, c
     are caller-owned outputs; nothing is allocated here.
     """
     _need_cuda(q, k, v, log_alpha, beta, S0, cu_seqlens, o, S_T)
-    shape = _shape_of(q, v, log_alpha, cu_seqlens, chunk, False)
+    shape = _shape_of(q, v, log_alpha, cu_seqlens, chunk, False, two_pass)
     rc = load_library().kda_chunk_fwd_noalloc(
         ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0),
         _ptr(cu_seqlens), _ptr(o), _ptr(S_T), _stream(stream))

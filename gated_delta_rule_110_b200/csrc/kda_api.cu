@@ -9,9 +9,10 @@
 #include <vector>
 
 #include "kda.h"
-#include "kda_chunk_fused.cuh"
 #include "kda_chunk_tc.cuh"
+#include "kda_prefill.cuh"
 #include "kda_recurrent.cuh"
+#include "kda_tma.h"
 
 namespace {
 
@@ -31,14 +32,16 @@ inline bool token_ptrs_aligned(const kda_shape& s, const void* q, const void* k,
 inline bool dtype_ok(int32_t d) { return d == KDA_F32 || d == KDA_BF16; }
 inline bool dim_ok(int32_t d) { return d == 64 || d == 128; }
 
-// Tensor-core chunk path: bf16 io, dk = dv = 128, C = 64.  It runs the fused
-// single-kernel form unless KDA_FLAG_PATH_TWO_PASS asks for the two-kernel
-// form (prep + recurrence through a workspace).
+// Tensor-core chunk path: bf16 io, dk = dv = 128, C = 64.  It runs the
+// pipelined kernel (state CTAs + transform CTAs through an L2-resident ring)
+// unless KDA_FLAG_PATH_TWO_PASS asks for the two-kernel form (prep + recurrence
+// through a workspace holding every chunk's operands).
 inline bool use_tc(const kda_shape& s) {
   return s.io_dtype == KDA_BF16 && s.dk == 128 && s.dv == 128 && s.chunk == 64;
 }
 inline bool use_two_pass(const kda_shape& s) { return use_tc(s) && (s.flags & KDA_FLAG_PATH_TWO_PASS) != 0u; }
-constexpr uint32_t kKnownFlags = KDA_FLAG_VALIDATE_CU_SEQLENS | KDA_FLAG_PATH_TWO_PASS;
+constexpr uint32_t kKnownFlags =
+    KDA_FLAG_VALIDATE_CU_SEQLENS | KDA_FLAG_PATH_TWO_PASS | KDA_FLAG_STATE_CTAS(0xFF) | KDA_FLAG_GRID_CTAS(0xFF);
 
 // Number of sequences N and the packed token total.
 inline void seq_counts(const kda_shape& s, const int32_t* cu, int64_t* N, int64_t* Ttot) {
@@ -146,17 +149,117 @@ kda_status launch_tc(const kda_shape& s, int64_t N, int64_t Ttot, const void* q,
   return launch_status();
 }
 
+// ---------------------------------------------------------------------------
+// Pipelined tensor-core prefill (kda_prefill.cuh)
+// ---------------------------------------------------------------------------
+int device_sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+struct PrefillPlan {
+  int R = 0;             // state CTAs
+  int grid = 0;          // all CTAs (one per SM)
+  size_t flag_bytes = 0; // zeroed before each launch
+  size_t ring_off = 0;
+  size_t bytes = 0;      // workspace
+};
+
+// Splits the SMs between state CTAs (one serial chain of chunks each) and
+// transform CTAs (parallel per-chunk work).  With `chains` (sequence, head)
+// pairs and a grid of G CTAs, R state CTAs take ceil(chains / R) chains each,
+// and the G - R transform CTAs share all chunks; a transform CTA needs about
+// kTransformCost times as long per chunk as a state CTA spends on one chunk
+// of its chain.  R minimises the larger of the two times.
+constexpr double kTransformCost = 2.0;
+
+PrefillPlan plan_prefill(const kda_shape& s, int64_t N, int nsm) {
+  PrefillPlan pl;
+  const int64_t chains = N * s.H;
+  int grid = nsm;
+  const int grid_req = static_cast<int>((s.flags >> 16) & 0xFFu);
+  if (grid_req > 0 && grid_req < grid) grid = grid_req;
+  if (grid < 2 || chains <= 0) return pl;
+  const int rmax = static_cast<int>(chains < grid - 1 ? chains : grid - 1);
+  int R = static_cast<int>((s.flags >> 8) & 0xFFu);
+  if (R > 0) {
+    R = R < rmax ? R : rmax;
+  } else {
+    double best = 1e300;
+    for (int r = 1; r <= rmax; ++r) {
+      const double t_state = static_cast<double>((chains + r - 1) / r);
+      const double t_tf = static_cast<double>(chains) * kTransformCost / (grid - r);
+      const double t = t_state > t_tf ? t_state : t_tf;
+      if (t < best - 1e-9) {
+        best = t;
+        R = r;
+      }
+    }
+  }
+  pl.R = R;
+  pl.grid = grid;
+  pl.flag_bytes = kda::pipe::flag_words(R) * sizeof(uint32_t);
+  pl.ring_off = (pl.flag_bytes + 1023) & ~static_cast<size_t>(1023);
+  pl.bytes = pl.ring_off + static_cast<size_t>(R) * kda::pipe::NRING * kda::pipe::SLOT;
+  return pl;
+}
+
 template <typename TG>
-kda_status launch_fused(const kda_shape& s, int64_t N, const void* q, const void* k, const void* v, const void* la,
-                        const void* beta, const float* S0, const int32_t* cu, void* o, float* S_T, cudaStream_t st) {
-  auto* kern = kda::fused::kda_chunk_fused_kernel<TG>;
-  if (!ensure_smem(kern, kda::fused::SMEM_BYTES)) return KDA_ERR_CUDA;
-  dim3 grid(static_cast<unsigned>(s.H), static_cast<unsigned>(N));
-  kern<<<grid, kda::fused::NTHREADS, kda::fused::SMEM_BYTES, st>>>(
-      s.T, s.H, cu, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-      static_cast<const __nv_bfloat16*>(v), static_cast<const TG*>(la), static_cast<const TG*>(beta), S0,
-      static_cast<__nv_bfloat16*>(o), S_T);
-  return launch_status();
+kda_status launch_prefill(const kda_shape& s, int64_t N, int64_t Ttot, const void* q, const void* k, const void* v,
+                          const void* la, const void* beta, const float* S0, const int32_t* cu, void* o, float* S_T,
+                          void* ws, size_t ws_bytes, cudaStream_t st) {
+  namespace P = kda::pipe;
+  const PrefillPlan pl = plan_prefill(s, N, device_sm_count());
+  if (pl.R <= 0) return KDA_ERR_CUDA;
+  if (!ws || ws_bytes < pl.bytes) return KDA_ERR_WORKSPACE;
+  // the work-item counter is 32-bit: R * (chunks of the longest stream) must fit
+  if (static_cast<double>(pl.R) * (static_cast<double>(Ttot) / P::C + static_cast<double>(N)) > 2.0e9)
+    return KDA_ERR_SHAPE;
+  P::Maps maps;
+  const uint64_t cols = static_cast<uint64_t>(s.H) * P::D;
+  const uint64_t rows = static_cast<uint64_t>(Ttot);
+  const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  bool ok = kda::make_tma_2d(&maps.q, q, bf, 2, cols, rows, cols * 2, 64, 64) &&
+            kda::make_tma_2d(&maps.k, k, bf, 2, cols, rows, cols * 2, 64, 64) &&
+            kda::make_tma_2d(&maps.v, v, bf, 2, cols, rows, cols * 2, 64, 64);
+  if (sizeof(TG) == 2)
+    ok = ok && kda::make_tma_2d(&maps.la, la, bf, 2, cols, rows, cols * 2, 64, 64);
+  else
+    ok = ok && kda::make_tma_2d(&maps.la, la, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, cols, rows, cols * 4, 32, 64);
+  if (!ok) return kda::tma_encode_fn() ? KDA_ERR_ALIGN : KDA_ERR_CUDA;
+  P::Params prm;
+  prm.T = s.T;
+  prm.H = s.H;
+  prm.N = static_cast<int>(N);
+  prm.R = pl.R;
+  prm.cu = cu;
+  prm.beta = beta;
+  prm.S0 = S0;
+  prm.o = static_cast<__nv_bfloat16*>(o);
+  prm.S_T = S_T;
+  prm.flags = static_cast<uint32_t*>(ws);
+  prm.ring = static_cast<uint8_t*>(ws) + pl.ring_off;
+  auto* kern = P::kda_prefill_kernel<TG>;
+  const uint32_t smem = P::ST_BYTES > P::TfLayout<TG>::BYTES ? P::ST_BYTES : P::TfLayout<TG>::BYTES;
+  if (!ensure_smem(kern, smem)) return KDA_ERR_CUDA;
+  if (cudaMemsetAsync(ws, 0, pl.flag_bytes, st) != cudaSuccess) return KDA_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(pl.grid));
+  cfg.blockDim = dim3(P::NTHREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, maps, prm) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return KDA_ERR_CUDA;
+  }
+  return KDA_OK;
 }
 
 kda_status validate_cu_host(const int32_t* cu, int64_t N, int64_t Ttot, cudaStream_t st) {
@@ -177,11 +280,12 @@ extern "C" {
 size_t kda_chunk_fwd_workspace_size(const kda_shape* sp) {
   if (check_common(sp) != KDA_OK) return 0;
   const kda_shape& s = *sp;
-  if (!use_two_pass(s)) return 0;
+  if (!use_tc(s)) return 0;
   const bool packed = s.n_seqs > 0 && s.B == 1;
   const int64_t N = packed ? s.n_seqs : s.B;
   const int64_t Ttot = packed ? s.T : static_cast<int64_t>(s.B) * s.T;
-  return static_cast<size_t>(max_chunks(N, Ttot)) * static_cast<size_t>(s.H) * SLOT_BYTES;
+  if (use_two_pass(s)) return static_cast<size_t>(max_chunks(N, Ttot)) * static_cast<size_t>(s.H) * SLOT_BYTES;
+  return plan_prefill(s, N, device_sm_count()).bytes;
 }
 
 kda_status kda_chunk_fwd(const kda_shape* sp, const void* q, const void* k, const void* v, const void* log_alpha,
@@ -206,10 +310,13 @@ kda_status kda_chunk_fwd(const kda_shape* sp, const void* q, const void* k, cons
   }
   if (N == 0) return KDA_OK;
 
-  if (use_tc(s) && !use_two_pass(s)) {
+  if (use_tc(s) && !use_two_pass(s) && Ttot > 0) {
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(log_alpha)) return KDA_ERR_ALIGN;
     if (s.gate_dtype == KDA_BF16)
-      return launch_fused<__nv_bfloat16>(s, N, q, k, v, log_alpha, beta, S0, cu_seqlens, o, S_T, st);
-    return launch_fused<float>(s, N, q, k, v, log_alpha, beta, S0, cu_seqlens, o, S_T, st);
+      return launch_prefill<__nv_bfloat16>(s, N, Ttot, q, k, v, log_alpha, beta, S0, cu_seqlens, o, S_T, workspace,
+                                           workspace_bytes, st);
+    return launch_prefill<float>(s, N, Ttot, q, k, v, log_alpha, beta, S0, cu_seqlens, o, S_T, workspace,
+                                 workspace_bytes, st);
   }
   if (use_two_pass(s)) {
     const size_t need = kda_chunk_fwd_workspace_size(sp);
@@ -313,11 +420,8 @@ extern "C" kda_status kda_chunk_fwd_noalloc(const kda_shape* sp_in, const void* 
                                             const int32_t* cu_seqlens, void* o, float* S_T, void* stream) {
   const kda_status e = check_common(sp_in);
   if (e != KDA_OK) return e;
-  // the two-pass kernels are the ones that need scratch; run them on the array
-  kda_shape shape = *sp_in;
-  shape.flags |= KDA_FLAG_PATH_TWO_PASS;
-  const kda_shape* sp = &shape;
-  // the size check needs no CUDA call, so an oversized request launches nothing
+  const kda_shape* sp = sp_in;
+  // an oversized request is refused before anything is launched
   const size_t need = kda_chunk_fwd_workspace_size(sp);
   if (need > kNoAllocScratchBytes) return KDA_ERR_WORKSPACE;
   void* scratch = nullptr;

@@ -1,0 +1,1115 @@
+// kda_prefill.cuh -- chunkwise-parallel KDA prefill on sm_100a as one
+// persistent, cooperatively launched kernel with two kinds of CTA.
+//
+// The chunk form ("Kimi Linear" summary page, section "Algoritmo paralelo por
+// chunks"): fixed chunks of C = 64 tokens, the final state of a chunk seeds the
+// next, the chunk's rank-1 updates are folded into a WY / UT representation
+// built with a lower-triangular inverse, and the output is an inter-chunk
+// (state) term plus an intra-chunk term.  The algebra, derived here from the
+// recurrence S_t = (I - b k k^T) Diag(a) S + b k v^T, o_t = S_t^T q_t, for a
+// chunk with rows r, g = per-channel cumulative log decay, a per-channel
+// reference ref = g_last / 2, sc = e^ref:
+//   Ka = K o e^{g - ref}   Qa = Q o e^{g - ref}   Kb = K o e^{ref - g}
+//   Kt = Kb Diag(sc) = K o e^{g_last - g}        gC = e^{g_last}
+//   A  = strict_tril(Diag(b) Ka Kb^T)           P = tril(Qa Kb^T)
+//   T  = (I + A)^-1,  Tb = T Diag(b),  W' = Tb Ka
+//   S' = Diag(sc) S        (S = state at the chunk start)
+//   U  = Tb V - W' S'      O = Qa S' + P U      S <- Diag(gC) S + Kt^T U
+// Everything above the line "S' = ..." is independent of the state, so it is
+// computed fully in parallel; only the last line is a chain over chunks.
+// Chunks whose total decay exceeds the factorised range (kSpan2, log2 units,
+// about 160 nats) take an exact CUDA-core A / P with sc = 1.
+//
+// CTA roles (grid = one CTA per SM, 384 threads, launched cooperatively so
+// every CTA is resident at once):
+//   * state CTAs (blockIdx < R) each own a stream of (sequence, head) chains
+//     and walk their chunks in order: the fp32 state S^T lives in registers of
+//     8 warps; bf16 copies of S'^T and U^T go to shared memory as MMA A
+//     operands; tcgen05 computes U^T, O^T and dS^T into TMEM.
+//   * transform CTAs (the rest) build the state-independent operands of one
+//     chunk at a time (two independent groups per CTA): cumulative log decay
+//     (a tensor-core product with a lower-triangular ones matrix), the scaled
+//     tiles, A / P on tcgen05, T by blocked forward substitution on CUDA cores,
+//     W'^T on tcgen05, and write them to a ring slot in global memory.
+// The ring (NRING slots per state CTA, ~65 KB each) is small enough to stay in
+// L2.  A transform CTA claims work items from a global counter in stream
+// order; it writes a slot once the state CTA has copied the slot's previous
+// contents (the `consumed` counter) and publishes it with a release store of
+// the position (`ready`).  The state CTA polls `ready` with acquire loads and
+// bulk-copies the slot into shared memory.  Items are claimed in increasing
+// stream position, so the smallest unfinished item can always proceed: with
+// every CTA resident the protocol cannot deadlock.  All waits are bounded; a
+// wait that runs out records KDA_ERR_TIMEOUT and raises a global abort flag
+// that every CTA polls.
+#pragma once
+
+#include "kda_ptx.cuh"
+
+namespace kda {
+namespace pipe {
+
+constexpr int C = 64;
+constexpr int D = 128;
+constexpr int NTHREADS = 384;
+constexpr int NRING = 4;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kSpan2 = 230.0f;  // largest chunk decay of the factorised path, log2 units
+
+// ---- ring slot: operands of one chunk as the state CTA's MMAs read them ----
+constexpr uint32_t R_TB = 0;       // Tb [r][s] bf16, K-major                     8 KB
+constexpr uint32_t R_WT = 8192;    // -W'^T [c][r] bf16, M/N-major B              16 KB
+constexpr uint32_t R_QA = 24576;   // Qa [r][c] bf16, two 64-channel atoms        16 KB
+constexpr uint32_t R_KT = 40960;   // Kt [r][c] bf16, two 64-channel atoms        16 KB
+constexpr uint32_t R_PP = 57344;   // P [r'][r] bf16, K-major                      8 KB
+constexpr uint32_t R_VEC = 65536;  // sc[128], gC[128] fp32                        1 KB
+constexpr uint32_t SLOT = 66560;
+
+// ---- global flags (32-bit words) ---------------------------------------------
+constexpr uint32_t F_COUNTER = 0;     // next work item
+constexpr uint32_t F_ABORT = 32;      // any CTA gave up
+constexpr uint32_t F_REC0 = 64;       // per state CTA: ready[NRING] at +0, consumed at +32
+constexpr uint32_t F_REC_STRIDE = 64;
+constexpr uint32_t F_CONSUMED = 32;
+__host__ __device__ constexpr size_t flag_words(int R) { return F_REC0 + static_cast<size_t>(R) * F_REC_STRIDE; }
+
+// ---- state CTA shared memory --------------------------------------------------
+constexpr uint32_t ST_SLOT = 0;                   // 2 ring slots
+constexpr uint32_t ST_V = 2 * SLOT;               // 2 x V tile [r][v] (two 64-value atoms)
+constexpr uint32_t ST_S = ST_V + 2 * 16384;       // S'^T [v][c] bf16, two 64-channel atoms
+constexpr uint32_t ST_U = ST_S + 32768;           // U^T [v][r] bf16
+constexpr uint32_t ST_BAR = ST_U + 16384;
+constexpr uint32_t ST_BYTES = ST_BAR + 256;
+// TMEM columns
+constexpr uint32_t TS_U = 0;     // U^T fp32        64
+constexpr uint32_t TS_DS = 128;  // dS^T fp32      128
+constexpr uint32_t TS_O = 256;   // 2 x O^T fp32    2 x 64
+
+// ---- transform CTA shared memory ------------------------------------------------
+template <typename TG>
+struct TfLayout {
+  static constexpr int NGROUP = sizeof(TG) == 2 ? 2 : 1;
+  static constexpr uint32_t RL_BYTES = sizeof(TG) == 2 ? 16384 : 32768;
+  static constexpr uint32_t L = 0;                       // [128][64] bf16 lower-triangular ones (twice)
+  static constexpr uint32_t G_RQ = 0;                    // raw q [r][c], two atoms
+  static constexpr uint32_t G_RK = 16384;                // raw k
+  static constexpr uint32_t G_RL = 32768;                // raw log-decay (bf16: 2 atoms, fp32: 4 atoms)
+  static constexpr uint32_t G_KQ = G_RL + RL_BYTES;      // [Ka; Qa] 2 K-atoms of [128][64]; T (fp32) later
+  static constexpr uint32_t G_KB = G_KQ + 32768;         // Kb 2 atoms of [64][64]; A (fp32) later
+  static constexpr uint32_t G_TB = G_KB + 16384;         // Tb [r][s]; inverse scratch before that
+  static constexpr uint32_t GROUP = G_TB + 8192;
+  static constexpr uint32_t GBASE = 16384;
+  static constexpr uint32_t MISC = GBASE + NGROUP * GROUP;
+  // per-group misc block
+  static constexpr uint32_t M_BETA = 0;     // fp32[64]
+  static constexpr uint32_t M_GL = 256;     // fp32[128]  g_last (log2 units)
+  static constexpr uint32_t M_SC = 768;     // fp32[128]  sc
+  static constexpr uint32_t M_META = 1280;  // int[16]
+  static constexpr uint32_t M_BAR = 1344;   // 16 mbarriers
+  static constexpr uint32_t MISC_GROUP = 1472;
+  static constexpr uint32_t BYTES = MISC + NGROUP * MISC_GROUP + 32;
+};
+// TMEM columns per transform group (group g at 256 g)
+constexpr uint32_t TT_G = 0;    // cumulative log decay [r][c] fp32 128
+constexpr uint32_t TT_AP = 128; // [A_raw; P_raw] fp32              64
+constexpr uint32_t TT_W = 192;  // W'^T fp32                        64
+
+// meta words
+enum { MT_DONE = 0, MT_SLOW, MT_N, MT_H, MT_J, MT_L, MT_I, MT_POS, MT_T0LO, MT_T0HI };
+// transform mbarriers
+enum { BT_RAW_FULL = 0, BT_RAW_FREE, BT_CS_GO, BT_CS_FULL, BT_AP_GO, BT_AP_FULL, BT_W_GO, BT_W_FULL, BT_FIN };
+// state mbarriers
+enum {
+  BS_SLOT_FULL = 0, BS_SLOT_FREE = 2, BS_S_READY = 4, BS_U_FULL, BS_U_READY, BS_DS_FULL, BS_O_FULL,
+  BS_O_FREE = BS_O_FULL + 2, BS_FIN = BS_O_FREE + 2, BS_COUNT
+};
+
+struct Params {
+  int T;            // tokens per batch row, or the packed total with cu
+  int H;            // heads
+  int N;            // sequences
+  int R;            // state CTAs
+  const int32_t* cu;
+  const void* beta;
+  const float* S0;
+  __nv_bfloat16* o;
+  float* S_T;
+  uint8_t* ring;    // R * NRING slots
+  uint32_t* flags;  // flag_words(R), zero on entry
+};
+
+struct Maps {
+  CUtensorMap q, k, v, la;
+};
+
+// --------------------------------------------------------------------------- helpers
+__device__ __forceinline__ void seq_range(const Params& p, int n, int64_t* b, int64_t* e) {
+  if (p.cu) {
+    *b = p.cu[n];
+    *e = p.cu[n + 1];
+  } else {
+    *b = static_cast<int64_t>(n) * p.T;
+    *e = *b + p.T;
+  }
+}
+__device__ __forceinline__ int seq_chunks(const Params& p, int n) {
+  int64_t b, e;
+  seq_range(p, n, &b, &e);
+  return static_cast<int>((e - b + C - 1) / C);
+}
+__device__ __forceinline__ int stream_len(const Params& p, int i) {
+  int len = 0;
+  for (int ci = i; ci < p.N * p.H; ci += p.R) len += seq_chunks(p, ci / p.H);
+  return len;
+}
+
+template <typename TG>
+__device__ __forceinline__ float ld_gate(const TG* ptr);
+template <>
+__device__ __forceinline__ float ld_gate<float>(const float* ptr) { return *ptr; }
+template <>
+__device__ __forceinline__ float ld_gate<__nv_bfloat16>(const __nv_bfloat16* ptr) { return __bfloat162float(*ptr); }
+
+__device__ __forceinline__ uint4 lds128(const uint8_t* p) { return *reinterpret_cast<const uint4*>(p); }
+__device__ __forceinline__ void sts128(uint8_t* p, uint4 x) { *reinterpret_cast<uint4*>(p) = x; }
+__device__ __forceinline__ void stg128(uint8_t* p, uint4 x) { *reinterpret_cast<uint4*>(p) = x; }
+__device__ __forceinline__ float2 bf2f(uint32_t u) {
+  __nv_bfloat162 b = *reinterpret_cast<__nv_bfloat162*>(&u);
+  return __bfloat1622float2(b);
+}
+
+// Polls a global counter until it reaches `target` (acquire).  Gives up when
+// the kernel-wide abort flag is raised or the wait runs out (then it raises
+// the flag itself and records KDA_ERR_TIMEOUT).
+__device__ __forceinline__ bool spin_geq(const uint32_t* flag, uint32_t target, uint32_t* gabort,
+                                         volatile int* abort_flag) {
+  if (ld_acquire_gpu(flag) >= target) return true;
+  const long long t0 = clock64();
+  for (uint32_t it = 0;; ++it) {
+    __nanosleep(64);
+    if (ld_acquire_gpu(flag) >= target) return true;
+    if ((it & 15u) == 15u) {
+      if (*abort_flag || *reinterpret_cast<volatile uint32_t*>(gabort) != 0u) {
+        *abort_flag = 1;
+        return false;
+      }
+      if (clock64() - t0 > kWaitCycles) {
+        record_error(-8 /* KDA_ERR_TIMEOUT */);
+        atomicExch(gabort, 1u);
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+
+// Element (r, s) of a 64 x 64 fp32 matrix whose 4-float groups are XOR-permuted
+// per row, so that 4 or 8 consecutive rows read at one column hit distinct banks.
+__device__ __forceinline__ int swzA(int r, int s) { return r * 64 + (s ^ ((((r & 7) ^ ((r >> 3) & 7))) << 2)); }
+
+// ===========================================================================
+// transform role: one group of 4 compute warps + a load warp + an MMA warp
+// ===========================================================================
+template <typename TG>
+struct Tf {
+  using LY = TfLayout<TG>;
+  uint8_t* smem;
+  uint32_t sbase;
+  uint8_t* gb;     // group base
+  uint32_t gba;    // group base (shared address)
+  uint8_t* misc;
+  uint64_t* bars;
+  int* meta;
+  uint32_t tmem;   // group TMEM base
+  int g;
+
+  __device__ Tf(uint8_t* sm, uint32_t tm, int grp) : smem(sm), g(grp) {
+    sbase = smem_u32(sm);
+    gb = sm + LY::GBASE + grp * LY::GROUP;
+    gba = sbase + LY::GBASE + grp * LY::GROUP;
+    misc = sm + LY::MISC + grp * LY::MISC_GROUP;
+    bars = reinterpret_cast<uint64_t*>(misc + LY::M_BAR);
+    meta = reinterpret_cast<int*>(misc + LY::M_META);
+    tmem = tm + 256u * grp;
+  }
+  __device__ float* betas() const { return reinterpret_cast<float*>(misc + LY::M_BETA); }
+  __device__ float* gls() const { return reinterpret_cast<float*>(misc + LY::M_GL); }
+  __device__ float* scs() const { return reinterpret_cast<float*>(misc + LY::M_SC); }
+  // T (fp32, [64][64]) lives in the Qa rows of the [Ka; Qa] tile once A/P is done
+  __device__ float* trow(int r) const {
+    return reinterpret_cast<float*>(gb + LY::G_KQ + (r < 32 ? 8192 : 24576) + (r & 31) * 256);
+  }
+  __device__ float* amat() const { return reinterpret_cast<float*>(gb + LY::G_KB); }
+  __device__ void bar() const { named_bar(1 + g, 128); }
+
+  // ------------------------------------------------------------ load warp
+  __device__ void load_loop(const Maps& maps, const Params& p, int maxlen, volatile int* abort_flag) {
+    const int lane = threadIdx.x & 31;
+    uint32_t* gflags = p.flags;
+    const long long total = static_cast<long long>(p.R) * maxlen;
+    int it = 0;
+    for (;; ++it) {
+      // lane 0 decides; every lane takes the same branch
+      int stop = 0, done = 0, i = 0, pos = 0, n = 0, h = 0, j = 0, L = 0;
+      int64_t t0 = 0;
+      if (lane == 0) {
+        if (it >= 1 && !mbar_wait(&bars[BT_RAW_FREE], (it - 1) & 1, abort_flag)) stop = 1;
+        while (!stop && !done) {
+          if (*abort_flag || *reinterpret_cast<volatile uint32_t*>(gflags + F_ABORT) != 0u) {
+            stop = 1;
+            break;
+          }
+          const long long w = atomicAdd(gflags + F_COUNTER, 1u);
+          if (w >= total) {
+            done = 1;
+            break;
+          }
+          i = static_cast<int>(w % p.R);
+          pos = static_cast<int>(w / p.R);
+          // walk state CTA i's chains to the chunk at stream position pos
+          int rem = pos;
+          bool found = false;
+          for (int ci = i; ci < p.N * p.H; ci += p.R) {
+            const int nc = seq_chunks(p, ci / p.H);
+            if (rem < nc) {
+              n = ci / p.H;
+              h = ci % p.H;
+              j = rem;
+              found = true;
+              break;
+            }
+            rem -= nc;
+          }
+          if (!found) continue;  // past the end of this stream
+          int64_t sb, se;
+          seq_range(p, n, &sb, &se);
+          t0 = sb + static_cast<int64_t>(j) * C;
+          L = static_cast<int>(se - t0 < C ? se - t0 : C);
+          break;
+        }
+      }
+      stop = __shfl_sync(0xffffffffu, stop, 0);
+      done = __shfl_sync(0xffffffffu, done, 0);
+      if (stop) break;
+      if (done) {
+        if (lane == 0) {
+          meta[MT_DONE] = 1;
+          mbar_arrive(&bars[BT_RAW_FULL]);
+        }
+        ++it;
+        break;
+      }
+      if (lane == 0) {
+        meta[MT_DONE] = 0;  // MT_SLOW belongs to the compute warps (the MMA warp may still read it)
+        meta[MT_N] = n;
+        meta[MT_H] = h;
+        meta[MT_J] = j;
+        meta[MT_L] = L;
+        meta[MT_I] = i;
+        meta[MT_POS] = pos;
+        meta[MT_T0LO] = static_cast<int>(static_cast<uint64_t>(t0) & 0xffffffffu);
+        meta[MT_T0HI] = static_cast<int>(static_cast<uint64_t>(t0) >> 32);
+        const int y = static_cast<int>(t0);
+        mbar_arrive_expect_tx(&bars[BT_RAW_FULL], 32768 + LY::RL_BYTES);
+        for (int hf = 0; hf < 2; ++hf) {
+          tma_load_2d(gb + LY::G_RQ + hf * 8192, &maps.q, h * D + 64 * hf, y, &bars[BT_RAW_FULL]);
+          tma_load_2d(gb + LY::G_RK + hf * 8192, &maps.k, h * D + 64 * hf, y, &bars[BT_RAW_FULL]);
+        }
+        if (sizeof(TG) == 2) {
+          for (int hf = 0; hf < 2; ++hf)
+            tma_load_2d(gb + LY::G_RL + hf * 8192, &maps.la, h * D + 64 * hf, y, &bars[BT_RAW_FULL]);
+        } else {
+          for (int qq = 0; qq < 4; ++qq)
+            tma_load_2d(gb + LY::G_RL + qq * 8192, &maps.la, h * D + 32 * qq, y, &bars[BT_RAW_FULL]);
+        }
+      }
+    }
+    // a load issued for an item that was never consumed must land before exit
+    if (lane == 0 && it >= 1) {
+      const long long t0 = clock64();
+      while (!mbar_try_wait(&bars[BT_RAW_FULL], (it - 1) & 1) && clock64() - t0 < kWaitCycles) {
+      }
+    }
+  }
+
+  // ------------------------------------------------------------- MMA warp
+  __device__ void mma_loop(volatile int* abort_flag) {
+    constexpr uint32_t id_cs = make_idesc_bf16(128, 128) | IDESC_B_MN;
+    constexpr uint32_t id_ap = make_idesc_bf16(128, 64);
+    constexpr uint32_t id_w = make_idesc_bf16(128, 64) | IDESC_A_MN;
+    const uint32_t Lb = sbase + LY::L;
+    for (int it = 0;; ++it) {
+      if (!mbar_wait(&bars[BT_CS_GO], it & 1, abort_flag)) break;
+      if (*reinterpret_cast<volatile int*>(&meta[MT_DONE])) break;
+      tc_fence_after();
+      if (sizeof(TG) == 2) {
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_bf16_ss(tmem + TT_G, make_sdesc_sw128(Lb + kk * 32, 16, 1024),
+                      make_sdesc_sw128(gba + LY::G_RL + kk * 2048, 8192, 1024), id_cs, kk > 0);
+      } else {
+        // log-decay split into three bf16 parts (in the KQ and KB areas)
+#pragma unroll
+        for (int t = 0; t < 3; ++t) {
+          const uint32_t base = gba + (t < 2 ? LY::G_KQ + 16384 * t : LY::G_KB);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16_ss(tmem + TT_G, make_sdesc_sw128(Lb + kk * 32, 16, 1024),
+                        make_sdesc_sw128(base + kk * 2048, 8192, 1024), id_cs, (t | kk) != 0);
+        }
+      }
+      mma_commit(&bars[BT_CS_FULL]);
+      if (!mbar_wait(&bars[BT_AP_GO], it & 1, abort_flag)) break;
+      tc_fence_after();
+      if (!*reinterpret_cast<volatile int*>(&meta[MT_SLOW])) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16_ss(tmem + TT_AP, make_sdesc_sw128(gba + LY::G_KQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                      make_sdesc_sw128(gba + LY::G_KB + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id_ap, kk > 0);
+      }
+      mma_commit(&bars[BT_AP_FULL]);
+      if (!mbar_wait(&bars[BT_W_GO], it & 1, abort_flag)) break;
+      tc_fence_after();
+      // W'^T [c][r] = sum_s Ka[s][c] Tb[r][s]  (A = Ka, M/N-major, channel atoms 16 KB apart)
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        mma_bf16_ss(tmem + TT_W, make_sdesc_sw128(gba + LY::G_KQ + kk * 2048, 16384, 1024),
+                    make_sdesc_sw128(gba + LY::G_TB + kk * 32, 16, 1024), id_w, kk > 0);
+      mma_commit(&bars[BT_W_FULL]);
+    }
+    mma_commit(&bars[BT_FIN]);
+    const long long t0 = clock64();
+    while (!mbar_try_wait(&bars[BT_FIN], 0) && clock64() - t0 < kWaitCycles) {
+    }
+  }
+
+  // --------------------------------------------------------- compute warps
+  __device__ void compute_loop(const Params& p, volatile int* abort_flag) {
+    const int gt = threadIdx.x - 128 * g;  // 0..127
+    const int q = gt >> 5, lane = gt & 31;
+    const int r = 32 * (q & 1) + lane;    // row of the elementwise / cumsum pass
+    const int ch = q >> 1;                // channel half
+    const uint32_t lane_off = static_cast<uint32_t>(32 * q) << 16;
+    uint32_t* gflags = p.flags;
+    float* sbeta = betas();
+    float* sgl = gls();
+    float* ssc = scs();
+    for (int it = 0;; ++it) {
+      // one decision for the whole group (its named barriers must stay matched):
+      // stop on completion or abort; inside the body a failed wait only raises
+      // the abort flag, and every barrier is still reached.
+      const bool got = mbar_wait_warp(&bars[BT_RAW_FULL], it & 1, abort_flag);
+      const bool fin = got && *reinterpret_cast<volatile int*>(&meta[MT_DONE]) != 0;
+      if (named_bar_or(1 + g, 128, !got || fin || *abort_flag)) {
+        if (gt == 0 && fin && !*abort_flag) mbar_arrive(&bars[BT_CS_GO]);
+        break;
+      }
+      const int L = meta[MT_L];
+      const int si = meta[MT_I];
+      const int pos = meta[MT_POS];
+      const int hh = meta[MT_H];
+      const int64_t t0 = static_cast<int64_t>((static_cast<uint64_t>(static_cast<uint32_t>(meta[MT_T0HI])) << 32) |
+                                              static_cast<uint32_t>(meta[MT_T0LO]));
+      uint8_t* slot = p.ring + (static_cast<size_t>(si) * NRING + (pos % NRING)) * SLOT;
+      // beta of this chunk (rows >= L are zero); the load overlaps the cumsum
+      // MMA, and the group owns its copy (the load warp moves on to the next
+      // chunk as soon as the raw tiles are released)
+      const float beta_r = gt < L ? ld_gate(static_cast<const TG*>(p.beta) + (t0 + gt) * p.H + hh) : 0.f;
+
+      // ---- C1: prepare the cumsum operand -------------------------------------
+      if (sizeof(TG) == 2) {
+        if (L < C) {
+          for (int e = gt; e < (C - L) * 16; e += 128) {
+            const int rr = L + (e >> 4), hf = (e >> 3) & 1, jj = e & 7;
+            sts128(gb + LY::G_RL + hf * 8192 + sw128(rr, jj), make_uint4(0u, 0u, 0u, 0u));
+          }
+        }
+      } else {
+        // split fp32 log-decay into hi + mid + lo bf16 tiles ([s][c], MN-major B)
+#pragma unroll 1
+        for (int jj = 0; jj < 8; ++jj) {
+          const int c0 = 64 * ch + 8 * jj;
+          float x[8];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int c = c0 + 4 * u;
+            const uint4 w = lds128(gb + LY::G_RL + (c >> 5) * 8192 + sw128(r, (c & 31) >> 2));
+            x[4 * u + 0] = __uint_as_float(w.x);
+            x[4 * u + 1] = __uint_as_float(w.y);
+            x[4 * u + 2] = __uint_as_float(w.z);
+            x[4 * u + 3] = __uint_as_float(w.w);
+          }
+          uint32_t pk[3][4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            float a0 = r < L ? x[2 * u] : 0.f, a1 = r < L ? x[2 * u + 1] : 0.f;
+            const float h0 = __bfloat162float(__float2bfloat16_rn(a0)), h1 = __bfloat162float(__float2bfloat16_rn(a1));
+            const float m0 = __bfloat162float(__float2bfloat16_rn(a0 - h0));
+            const float m1 = __bfloat162float(__float2bfloat16_rn(a1 - h1));
+            pk[0][u] = pack_bf16(h0, h1);
+            pk[1][u] = pack_bf16(m0, m1);
+            pk[2][u] = pack_bf16(a0 - h0 - m0, a1 - h1 - m1);
+          }
+#pragma unroll
+          for (int t = 0; t < 3; ++t) {
+            uint8_t* base = gb + (t < 2 ? LY::G_KQ + 16384 * t : LY::G_KB);
+            sts128(base + ch * 8192 + sw128(r, jj), make_uint4(pk[t][0], pk[t][1], pk[t][2], pk[t][3]));
+          }
+        }
+      }
+      fence_proxy_async_smem();
+      bar();
+      if (gt == 0) mbar_arrive(&bars[BT_CS_GO]);
+
+      // ---- C2: cumulative decay -> scaled tiles ---------------------------------
+      if (gt < C) sbeta[gt] = beta_r;  // published by the barriers below
+      mbar_wait_warp(&bars[BT_CS_FULL], it & 1, abort_flag);
+      tc_fence_after();
+      float g2[64];
+      {
+        float x[32];
+        tmem_ld32(tmem + lane_off + TT_G + 64 * ch, x);
+        tmem_wait_ld();
+#pragma unroll
+        for (int u = 0; u < 32; ++u) g2[u] = x[u] * kLog2e;
+        tmem_ld32(tmem + lane_off + TT_G + 64 * ch + 32, x);
+        tmem_wait_ld();
+#pragma unroll
+        for (int u = 0; u < 32; ++u) g2[32 + u] = x[u] * kLog2e;
+      }
+      bool steep = false;  // this thread holds row 63 and a channel decays beyond the factorised range
+      if ((q & 1) && lane == 31) {
+#pragma unroll
+        for (int u = 0; u < 64; ++u) {
+          sgl[64 * ch + u] = g2[u];
+          steep = steep || (-g2[u] > kSpan2);
+        }
+      }
+      // the ring slot must have been copied out by its state CTA
+      if (gt == 0 && pos + 1 - NRING > 0)
+        spin_geq(gflags + F_REC0 + si * F_REC_STRIDE + F_CONSUMED, static_cast<uint32_t>(pos + 1 - NRING),
+                 gflags + F_ABORT, abort_flag);
+      const bool slow = named_bar_or(1 + g, 128, steep);
+      {
+        // per channel: sc = 2^{g_last/2} (1 on the exact path), gamma_C = 2^{g_last}
+        const float gl = sgl[gt];
+        const float sc = slow ? 1.f : ex2_approx(0.5f * gl);
+        ssc[gt] = sc;
+        float* vec = reinterpret_cast<float*>(slot + R_VEC);
+        vec[gt] = sc;
+        vec[128 + gt] = ex2_approx(gl);
+      }
+      bar();
+      if (!slow) {
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          const int c0 = 64 * ch + 8 * jj;
+          uint4 kw = lds128(gb + LY::G_RK + ch * 8192 + sw128(r, jj));
+          uint4 qw = lds128(gb + LY::G_RQ + ch * 8192 + sw128(r, jj));
+          if (r >= L) kw = qw = make_uint4(0u, 0u, 0u, 0u);
+          const uint32_t kk4[4] = {kw.x, kw.y, kw.z, kw.w}, qq4[4] = {qw.x, qw.y, qw.z, qw.w};
+          uint32_t ka[4], qa[4], kb[4], kt[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int c = c0 + 2 * u;
+            const float2 kx = bf2f(kk4[u]), qx = bf2f(qq4[u]);
+            const float rf0 = 0.5f * sgl[c], rf1 = 0.5f * sgl[c + 1];
+            const float x0 = g2[8 * jj + 2 * u], x1 = g2[8 * jj + 2 * u + 1];
+            const float e10 = ex2_approx(x0 - rf0), e11 = ex2_approx(x1 - rf1);
+            const float e20 = ex2_approx(rf0 - x0), e21 = ex2_approx(rf1 - x1);
+            ka[u] = pack_bf16(kx.x * e10, kx.y * e11);
+            qa[u] = pack_bf16(qx.x * e10, qx.y * e11);
+            const float b0 = kx.x * e20, b1 = kx.y * e21;
+            kb[u] = pack_bf16(b0, b1);
+            kt[u] = pack_bf16(b0 * ssc[c], b1 * ssc[c + 1]);
+          }
+          const uint4 kav = make_uint4(ka[0], ka[1], ka[2], ka[3]), qav = make_uint4(qa[0], qa[1], qa[2], qa[3]);
+          sts128(gb + LY::G_KQ + ch * 16384 + sw128(r, jj), kav);
+          sts128(gb + LY::G_KQ + ch * 16384 + sw128(64 + r, jj), qav);
+          sts128(gb + LY::G_KB + ch * 8192 + sw128(r, jj), make_uint4(kb[0], kb[1], kb[2], kb[3]));
+          stg128(slot + R_QA + ch * 8192 + sw128(r, jj), qav);
+          stg128(slot + R_KT + ch * 8192 + sw128(r, jj), make_uint4(kt[0], kt[1], kt[2], kt[3]));
+        }
+      } else {
+        // ---- exact path: A and P term by term from g (fp32, in the KQ area) ------
+        float* G = reinterpret_cast<float*>(gb + LY::G_KQ);
+#pragma unroll
+        for (int u = 0; u < 64; u += 4)
+          *reinterpret_cast<float4*>(G + r * 128 + 64 * ch + u) = make_float4(g2[u], g2[u + 1], g2[u + 2], g2[u + 3]);
+        bar();
+        const uint8_t* RK = gb + LY::G_RK;
+        const uint8_t* RQ = gb + LY::G_RQ;
+        auto kval = [&](const uint8_t* tile, int row, int c) -> float {
+          const uint16_t raw = *reinterpret_cast<const uint16_t*>(tile + (c >> 6) * 8192 + sw128(row, (c & 63) >> 3) +
+                                                                  (c & 7) * 2);
+          return row < L ? __bfloat162float(__ushort_as_bfloat16(raw)) : 0.f;
+        };
+        float* Af = amat();
+#pragma unroll 1
+        for (int e = gt; e < C * C; e += 128) {
+          const int ar = e >> 6, as = e & 63;
+          float a = 0.f, pp = 0.f;
+          if (as <= ar) {
+#pragma unroll 4
+            for (int c = 0; c < D; ++c) {
+              const float ex = ex2_approx(G[ar * 128 + c] - G[as * 128 + c]);
+              const float kse = kval(RK, as, c) * ex;
+              a += kval(RK, ar, c) * kse;
+              pp += kval(RQ, ar, c) * kse;
+            }
+          }
+          Af[swzA(ar, as)] = as < ar ? sbeta[ar] * a : 0.f;
+          *reinterpret_cast<__nv_bfloat16*>(slot + R_PP + sw128(ar, as >> 3) + (as & 7) * 2) = __float2bfloat16_rn(pp);
+        }
+        bar();  // g is dead; Ka / Qa overwrite it
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          const int c0 = 64 * ch + 8 * jj;
+          uint4 kw = lds128(gb + LY::G_RK + ch * 8192 + sw128(r, jj));
+          uint4 qw = lds128(gb + LY::G_RQ + ch * 8192 + sw128(r, jj));
+          if (r >= L) kw = qw = make_uint4(0u, 0u, 0u, 0u);
+          const uint32_t kk4[4] = {kw.x, kw.y, kw.z, kw.w}, qq4[4] = {qw.x, qw.y, qw.z, qw.w};
+          uint32_t ka[4], qa[4], kt[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int c = c0 + 2 * u;
+            const float2 kx = bf2f(kk4[u]), qx = bf2f(qq4[u]);
+            const float x0 = g2[8 * jj + 2 * u], x1 = g2[8 * jj + 2 * u + 1];
+            const float gm0 = ex2_approx(x0), gm1 = ex2_approx(x1);
+            const float ps0 = ex2_approx(sgl[c] - x0), ps1 = ex2_approx(sgl[c + 1] - x1);
+            ka[u] = pack_bf16(kx.x * gm0, kx.y * gm1);
+            qa[u] = pack_bf16(qx.x * gm0, qx.y * gm1);
+            kt[u] = pack_bf16(kx.x * ps0, kx.y * ps1);
+          }
+          const uint4 kav = make_uint4(ka[0], ka[1], ka[2], ka[3]), qav = make_uint4(qa[0], qa[1], qa[2], qa[3]);
+          sts128(gb + LY::G_KQ + ch * 16384 + sw128(r, jj), kav);
+          sts128(gb + LY::G_KQ + ch * 16384 + sw128(64 + r, jj), qav);
+          stg128(slot + R_QA + ch * 8192 + sw128(r, jj), qav);
+          stg128(slot + R_KT + ch * 8192 + sw128(r, jj), make_uint4(kt[0], kt[1], kt[2], kt[3]));
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      bar();
+      if (gt == 0) {
+        meta[MT_SLOW] = slow ? 1 : 0;
+        mbar_arrive(&bars[BT_RAW_FREE]);
+        mbar_arrive(&bars[BT_AP_GO]);
+      }
+
+      // ---- C3: A / P epilogue -------------------------------------------------------
+      mbar_wait_warp(&bars[BT_AP_FULL], it & 1, abort_flag);
+      tc_fence_after();
+      if (!slow) {
+        float x[64];
+        {
+          float t[32];
+          tmem_ld32(tmem + lane_off + TT_AP, t);
+          tmem_wait_ld();
+#pragma unroll
+          for (int u = 0; u < 32; ++u) x[u] = t[u];
+          tmem_ld32(tmem + lane_off + TT_AP + 32, t);
+          tmem_wait_ld();
+#pragma unroll
+          for (int u = 0; u < 32; ++u) x[32 + u] = t[u];
+        }
+        if (q < 2) {
+          const int ar = 32 * q + lane;
+          const float br = sbeta[ar];
+          float* Af = amat();
+#pragma unroll
+          for (int s4 = 0; s4 < 16; ++s4) {
+            float4 w;
+            w.x = 4 * s4 + 0 < ar ? br * x[4 * s4 + 0] : 0.f;
+            w.y = 4 * s4 + 1 < ar ? br * x[4 * s4 + 1] : 0.f;
+            w.z = 4 * s4 + 2 < ar ? br * x[4 * s4 + 2] : 0.f;
+            w.w = 4 * s4 + 3 < ar ? br * x[4 * s4 + 3] : 0.f;
+            *reinterpret_cast<float4*>(Af + swzA(ar, 4 * s4)) = w;
+          }
+        } else {
+          const int rp = 32 * (q - 2) + lane;
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj) {
+            uint32_t pk[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int s0 = 8 * jj + 2 * u;
+              pk[u] = pack_bf16(s0 <= rp ? x[s0] : 0.f, s0 + 1 <= rp ? x[s0 + 1] : 0.f);
+            }
+            stg128(slot + R_PP + sw128(rp, jj), make_uint4(pk[0], pk[1], pk[2], pk[3]));
+          }
+        }
+      }
+      bar();
+
+      // ---- C4: T = (I + A)^-1, blocked forward substitution (fp32) ---------------
+      invert(sbeta);
+      // Tb = T Diag(beta) -> bf16 [r][s] (local MMA operand and ring slot)
+      {
+        const int tr = gt >> 1, sh = gt & 1;
+        const float* Tr = trow(tr);
+#pragma unroll
+        for (int j4 = 0; j4 < 4; ++j4) {
+          const int s0 = 32 * sh + 8 * j4;
+          uint32_t pk[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int s = s0 + 2 * u;
+            const float a = (s >> 4) <= (tr >> 4) ? Tr[s] * sbeta[s] : 0.f;
+            const float b = ((s + 1) >> 4) <= (tr >> 4) ? Tr[s + 1] * sbeta[s + 1] : 0.f;
+            pk[u] = pack_bf16(a, b);
+          }
+          const uint4 w = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          sts128(gb + LY::G_TB + sw128(tr, s0 >> 3), w);
+          stg128(slot + R_TB + sw128(tr, s0 >> 3), w);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      bar();
+      if (gt == 0) mbar_arrive(&bars[BT_W_GO]);
+
+      // ---- C5: -W'^T -> ring slot, then publish --------------------------------------
+      mbar_wait_warp(&bars[BT_W_FULL], it & 1, abort_flag);
+      tc_fence_after();
+      {
+        const int c = 32 * q + lane;
+        float x[32];
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          tmem_ld32(tmem + lane_off + TT_W + 32 * hf, x);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j4 = 0; j4 < 4; ++j4) {
+            uint32_t pk[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) pk[u] = pack_bf16(-x[8 * j4 + 2 * u], -x[8 * j4 + 2 * u + 1]);
+            stg128(slot + R_WT + sw128(c, 4 * hf + j4), make_uint4(pk[0], pk[1], pk[2], pk[3]));
+          }
+        }
+      }
+      tc_fence_before();
+      bar();
+      if (gt == 0 && !*abort_flag) {
+        __threadfence();
+        st_release_gpu(gflags + F_REC0 + si * F_REC_STRIDE + (pos % NRING), static_cast<uint32_t>(pos + 1));
+      }
+    }
+  }
+
+  // T = (I + A)^-1 for the strictly lower-triangular A (fp32, swizzled rows in
+  // the KB area), written to trow().  Diagonal 16 x 16 blocks by column-wise
+  // forward substitution; then block levels d = 1, 2, 3:
+  //   T_IJ = -T_II sum_{K=J}^{I-1} A_IK T_KJ      (I - J = d)
+  __device__ void invert(const float* sbeta) {
+    const int gt = threadIdx.x - 128 * g;
+    const float* Af = amat();
+    float* X = reinterpret_cast<float*>(gb + LY::G_TB);  // scratch, [3][16][16]
+    if (gt < 64) {
+      const int I = gt >> 4, jc = gt & 15;
+      float x[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) x[i] = i == jc ? 1.f : 0.f;
+#pragma unroll
+      for (int m = 0; m < 15; ++m) {
+        const float xm = x[m];
+#pragma unroll
+        for (int i = m + 1; i < 16; ++i) x[i] -= Af[swzA(16 * I + i, 16 * I + m)] * xm;
+      }
+#pragma unroll
+      for (int i = 0; i < 16; ++i) trow(16 * I + i)[16 * I + jc] = x[i];
+    }
+    bar();
+    const int i = gt >> 3, j = 2 * (gt & 7);  // each thread: row i, columns j, j+1 of a 16 x 16 block
+    for (int d = 1; d < 4; ++d) {
+      const int nb = 4 - d;
+      for (int b = 0; b < nb; ++b) {
+        const int I = b + d, J = b;
+        float a0 = 0.f, a1 = 0.f;
+        for (int K = J; K < I; ++K) {
+#pragma unroll
+          for (int m = 0; m < 16; ++m) {
+            const float av = Af[swzA(16 * I + i, 16 * K + m)];
+            const float2 tv = *reinterpret_cast<const float2*>(trow(16 * K + m) + 16 * J + j);
+            a0 += av * tv.x;
+            a1 += av * tv.y;
+          }
+        }
+        *reinterpret_cast<float2*>(X + (b * 16 + i) * 16 + j) = make_float2(a0, a1);
+      }
+      bar();
+      for (int b = 0; b < nb; ++b) {
+        const int I = b + d, J = b;
+        float a0 = 0.f, a1 = 0.f;
+        const float* Ti = trow(16 * I + i);
+#pragma unroll
+        for (int m = 0; m < 16; ++m) {
+          const float tv = Ti[16 * I + m];
+          const float2 xv = *reinterpret_cast<const float2*>(X + (b * 16 + m) * 16 + j);
+          a0 += tv * xv.x;
+          a1 += tv * xv.y;
+        }
+        *reinterpret_cast<float2*>(trow(16 * I + i) + 16 * J + j) = make_float2(-a0, -a1);
+      }
+      bar();
+    }
+  }
+};
+
+// ===========================================================================
+// state role
+// ===========================================================================
+struct StateWalk {
+  int ci, nc;
+  int64_t sb, se;
+  __device__ bool next(const Params& p) {
+    ci += p.R;
+    if (ci >= p.N * p.H) return false;
+    seq_range(p, ci / p.H, &sb, &se);
+    nc = static_cast<int>((se - sb + C - 1) / C);
+    return true;
+  }
+};
+
+__device__ __forceinline__ void state_load_loop(uint8_t* smem, const Maps& maps, const Params& p, uint64_t* bars,
+                                                volatile int* abort_flag) {
+  const int i = blockIdx.x;
+  uint32_t* gflags = p.flags;
+  const uint32_t* ready = gflags + F_REC0 + i * F_REC_STRIDE;
+  uint32_t* consumed = gflags + F_REC0 + i * F_REC_STRIDE + F_CONSUMED;
+  int pos = 0;
+  bool ok = true;
+  StateWalk w{i - p.R, 0, 0, 0};
+  while (ok && w.next(p)) {
+    const int h = w.ci % p.H;
+    for (int j = 0; j < w.nc; ++j, ++pos) {
+      const int s = pos & 1;
+      if (pos >= 2 && !mbar_wait(&bars[BS_SLOT_FREE + s], ((pos - 2) >> 1) & 1, abort_flag)) {
+        ok = false;
+        break;
+      }
+      if (!spin_geq(ready + (pos % NRING), static_cast<uint32_t>(pos + 1), gflags + F_ABORT, abort_flag)) {
+        ok = false;
+        break;
+      }
+      fence_proxy_async_global();
+      const int64_t t0 = w.sb + static_cast<int64_t>(j) * C;
+      mbar_arrive_expect_tx(&bars[BS_SLOT_FULL + s], SLOT + 16384);
+      const uint8_t* src = p.ring + (static_cast<size_t>(i) * NRING + (pos % NRING)) * SLOT;
+      uint8_t* dst = smem + ST_SLOT + s * SLOT;
+      bulk_g2s(dst, src, 32768, &bars[BS_SLOT_FULL + s]);
+      bulk_g2s(dst + 32768, src + 32768, SLOT - 32768, &bars[BS_SLOT_FULL + s]);
+      for (int hf = 0; hf < 2; ++hf)
+        tma_load_2d(smem + ST_V + s * 16384 + hf * 8192, &maps.v, h * D + 64 * hf, static_cast<int>(t0),
+                    &bars[BS_SLOT_FULL + s]);
+      // the previous position's copy has landed: its ring slot may be reused
+      if (pos >= 1) {
+        const int pp = pos - 1;
+        if (!mbar_wait(&bars[BS_SLOT_FULL + (pp & 1)], (pp >> 1) & 1, abort_flag)) {
+          ok = false;
+          ++pos;
+          break;
+        }
+        fence_proxy_async_global();
+        st_release_gpu(consumed, static_cast<uint32_t>(pos));
+      }
+    }
+  }
+  // drain: copies still landing in shared memory must finish before exit
+  for (int pp = pos - 2 < 0 ? 0 : pos - 2; pp < pos; ++pp) {
+    const long long t0 = clock64();
+    while (!mbar_try_wait(&bars[BS_SLOT_FULL + (pp & 1)], (pp >> 1) & 1) && clock64() - t0 < kWaitCycles) {
+    }
+  }
+}
+
+__device__ __forceinline__ void state_mma_loop(uint32_t sbase, uint32_t tmem, const Params& p, uint64_t* bars,
+                                               volatile int* abort_flag) {
+  constexpr uint32_t id_uv = make_idesc_bf16(128, 64) | IDESC_A_MN;
+  constexpr uint32_t id_us = make_idesc_bf16(128, 64) | IDESC_B_MN;
+  constexpr uint32_t id_n64 = make_idesc_bf16(128, 64);
+  constexpr uint32_t id_ds = make_idesc_bf16(128, 128) | IDESC_B_MN;
+  const int i = blockIdx.x;
+  int pos = 0;
+  bool ok = true;
+  StateWalk w{i - p.R, 0, 0, 0};
+  while (ok && w.next(p)) {
+    for (int j = 0; j < w.nc; ++j, ++pos) {
+      const int s = pos & 1, b = pos & 1;
+      const uint32_t slot = sbase + ST_SLOT + s * SLOT;
+      const uint32_t vt = sbase + ST_V + s * 16384;
+      if (!mbar_wait(&bars[BS_SLOT_FULL + s], (pos >> 1) & 1, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      // U^T = V^T Tb^T
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        mma_bf16_ss(tmem + TS_U, make_sdesc_sw128(vt + kk * 2048, 8192, 1024),
+                    make_sdesc_sw128(slot + R_TB + kk * 32, 16, 1024), id_uv, kk > 0);
+      if (!mbar_wait(&bars[BS_S_READY], pos & 1, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      // U^T += S'^T (-W'^T)
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        mma_bf16_ss(tmem + TS_U, make_sdesc_sw128(sbase + ST_S + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                    make_sdesc_sw128(slot + R_WT + kk * 2048, 8192, 1024), id_us, 1);
+      mma_commit(&bars[BS_U_FULL]);
+      // O^T = S'^T Qa^T  (buffer b, free once position pos-2 was read out)
+      if (pos >= 2 && !mbar_wait(&bars[BS_O_FREE + b], ((pos - 2) >> 1) & 1, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        mma_bf16_ss(tmem + TS_O + 64 * b,
+                    make_sdesc_sw128(sbase + ST_S + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                    make_sdesc_sw128(slot + R_QA + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id_n64, kk > 0);
+      if (!mbar_wait(&bars[BS_U_READY], pos & 1, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      // dS^T = U^T Kt
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        mma_bf16_ss(tmem + TS_DS, make_sdesc_sw128(sbase + ST_U + kk * 32, 16, 1024),
+                    make_sdesc_sw128(slot + R_KT + kk * 2048, 8192, 1024), id_ds, kk > 0);
+      mma_commit(&bars[BS_DS_FULL]);
+      // O^T += U^T P^T
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        mma_bf16_ss(tmem + TS_O + 64 * b, make_sdesc_sw128(sbase + ST_U + kk * 32, 16, 1024),
+                    make_sdesc_sw128(slot + R_PP + kk * 32, 16, 1024), id_n64, 1);
+      mma_commit(&bars[BS_O_FULL + b]);
+      mma_commit(&bars[BS_SLOT_FREE + s]);
+    }
+    if (!ok) break;
+  }
+  mma_commit(&bars[BS_FIN]);
+  const long long t0 = clock64();
+  while (!mbar_try_wait(&bars[BS_FIN], 0) && clock64() - t0 < kWaitCycles) {
+  }
+}
+
+// 8 warps; thread (q = warp & 3, hf = warp >> 2) owns value column v = 32 q + lane
+// and channels [64 hf, 64 hf + 64) of S^T, in registers.
+__device__ __forceinline__ void state_warps_loop(uint8_t* smem, uint32_t tmem, const Params& p, uint64_t* bars,
+                                                 volatile int* abort_flag) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int q = warp & 3, hf = warp >> 2;
+  const int v = 32 * q + lane;
+  const uint32_t lane_off = static_cast<uint32_t>(32 * q) << 16;
+  const int i = blockIdx.x;
+  float S[64];
+  int pos = 0;
+  bool ok = true;
+  // output of the previous position, read out one step late
+  int prev_L = 0, prev_h = 0;
+  int64_t prev_t0 = 0;
+  bool have_prev = false;
+
+  auto o_pass = [&](int pp) -> bool {
+    const int b = pp & 1;
+    if (!mbar_wait_warp(&bars[BS_O_FULL + b], (pp >> 1) & 1, abort_flag)) return false;
+    tc_fence_after();
+    float x[32];
+    tmem_ld32(tmem + lane_off + TS_O + 64 * b + 32 * hf, x);
+    tmem_wait_ld();
+    tc_fence_before();
+    mbar_arrive(&bars[BS_O_FREE + b]);
+    __nv_bfloat16* op = p.o + (prev_t0 * p.H + prev_h) * D + v;
+#pragma unroll
+    for (int u = 0; u < 32; ++u) {
+      const int rr = 32 * hf + u;
+      if (rr < prev_L) op[static_cast<int64_t>(rr) * p.H * D] = __float2bfloat16_rn(x[u]);
+    }
+    return true;
+  };
+
+  StateWalk w{i - p.R, 0, 0, 0};
+  while (ok && w.next(p)) {
+    const int n = w.ci / p.H, h = w.ci % p.H;
+    const size_t sidx = (static_cast<size_t>(n) * p.H + h) * D * D;
+    if (p.S0) {
+#pragma unroll
+      for (int u = 0; u < 64; ++u) S[u] = p.S0[sidx + static_cast<size_t>(64 * hf + u) * D + v];
+    } else {
+#pragma unroll
+      for (int u = 0; u < 64; ++u) S[u] = 0.f;
+    }
+    for (int j = 0; j < w.nc; ++j, ++pos) {
+      const int s = pos & 1;
+      const uint8_t* slot = smem + ST_SLOT + s * SLOT;
+      if (!mbar_wait_warp(&bars[BS_SLOT_FULL + s], (pos >> 1) & 1, abort_flag)) { ok = false; break; }
+      // S'^T = bf16(sc S^T) -> shared memory (A operand); S <- gamma_C S
+      {
+        const float* sc = reinterpret_cast<const float*>(slot + R_VEC) + 64 * hf;
+        const float* gc = reinterpret_cast<const float*>(slot + R_VEC) + 128 + 64 * hf;
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          uint32_t pk[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int c = 8 * jj + 2 * u;
+            pk[u] = pack_bf16(S[c] * sc[c], S[c + 1] * sc[c + 1]);
+          }
+          sts128(smem + ST_S + hf * 16384 + sw128(v, jj), make_uint4(pk[0], pk[1], pk[2], pk[3]));
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&bars[BS_S_READY]);
+#pragma unroll
+        for (int u = 0; u < 64; ++u) S[u] *= gc[u];
+      }
+      if (have_prev && !o_pass(pos - 1)) { ok = false; break; }
+      // U^T -> bf16 shared memory (A operand)
+      if (!mbar_wait_warp(&bars[BS_U_FULL], pos & 1, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      {
+        float x[32];
+        tmem_ld32(tmem + lane_off + TS_U + 32 * hf, x);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j4 = 0; j4 < 4; ++j4) {
+          uint32_t pk[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) pk[u] = pack_bf16(x[8 * j4 + 2 * u], x[8 * j4 + 2 * u + 1]);
+          sts128(smem + ST_U + sw128(v, 4 * hf + j4), make_uint4(pk[0], pk[1], pk[2], pk[3]));
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&bars[BS_U_READY]);
+      // S += dS
+      if (!mbar_wait_warp(&bars[BS_DS_FULL], pos & 1, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      {
+        float x[32];
+        tmem_ld32(tmem + lane_off + TS_DS + 64 * hf, x);
+        tmem_wait_ld();
+#pragma unroll
+        for (int u = 0; u < 32; ++u) S[u] += x[u];
+        tmem_ld32(tmem + lane_off + TS_DS + 64 * hf + 32, x);
+        tmem_wait_ld();
+#pragma unroll
+        for (int u = 0; u < 32; ++u) S[32 + u] += x[u];
+      }
+      tc_fence_before();
+      const int64_t t0 = w.sb + static_cast<int64_t>(j) * C;
+      prev_t0 = t0;
+      prev_h = h;
+      prev_L = static_cast<int>(w.se - t0 < C ? w.se - t0 : C);
+      have_prev = true;
+    }
+    if (!ok) break;
+    if (p.S_T) {
+#pragma unroll
+      for (int u = 0; u < 64; ++u) p.S_T[sidx + static_cast<size_t>(64 * hf + u) * D + v] = S[u];
+    }
+  }
+  if (ok && have_prev) o_pass(pos - 1);
+}
+
+// ===========================================================================
+// the kernel
+// ===========================================================================
+template <typename TG>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    kda_prefill_kernel(const __grid_constant__ Maps maps, const Params p) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  using LY = TfLayout<TG>;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool is_state = static_cast<int>(blockIdx.x) < p.R;
+  const uint32_t sbase = smem_u32(smem);
+  uint64_t* bars;
+  uint32_t* tmem_slot;
+  volatile int* abort_flag;
+  int* s_maxlen = nullptr;  // transform CTAs: longest stream of any state CTA
+  if (is_state) {
+    bars = reinterpret_cast<uint64_t*>(smem + ST_BAR);
+    tmem_slot = reinterpret_cast<uint32_t*>(smem + ST_BAR + 8 * BS_COUNT);
+    abort_flag = reinterpret_cast<volatile int*>(smem + ST_BAR + 8 * BS_COUNT + 8);
+  } else {
+    bars = reinterpret_cast<uint64_t*>(smem + LY::MISC + LY::M_BAR);
+    tmem_slot = reinterpret_cast<uint32_t*>(smem + LY::MISC + LY::NGROUP * LY::MISC_GROUP);
+    abort_flag = reinterpret_cast<volatile int*>(smem + LY::MISC + LY::NGROUP * LY::MISC_GROUP + 8);
+    s_maxlen = reinterpret_cast<int*>(smem + LY::MISC + LY::NGROUP * LY::MISC_GROUP + 16);
+  }
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    if (!is_state) *s_maxlen = 0;
+    if (is_state) {
+      mbar_init(&bars[BS_SLOT_FULL + 0], 1);
+      mbar_init(&bars[BS_SLOT_FULL + 1], 1);
+      mbar_init(&bars[BS_SLOT_FREE + 0], 1);
+      mbar_init(&bars[BS_SLOT_FREE + 1], 1);
+      mbar_init(&bars[BS_S_READY], 256);
+      mbar_init(&bars[BS_U_FULL], 1);
+      mbar_init(&bars[BS_U_READY], 256);
+      mbar_init(&bars[BS_DS_FULL], 1);
+      mbar_init(&bars[BS_O_FULL + 0], 1);
+      mbar_init(&bars[BS_O_FULL + 1], 1);
+      mbar_init(&bars[BS_O_FREE + 0], 256);
+      mbar_init(&bars[BS_O_FREE + 1], 256);
+      mbar_init(&bars[BS_FIN], 1);
+    } else {
+      for (int g = 0; g < LY::NGROUP; ++g) {
+        uint64_t* gbars = reinterpret_cast<uint64_t*>(smem + LY::MISC + g * LY::MISC_GROUP + LY::M_BAR);
+        for (int b = 0; b <= BT_FIN; ++b) mbar_init(&gbars[b], 1);
+      }
+    }
+    fence_mbar_init();
+  }
+  if (!is_state) {
+    // the cumsum operand [L; L], L[r][s] = (s <= r), bf16, K-major
+    for (int e = threadIdx.x; e < 128 * 8; e += NTHREADS) {
+      const int rr = e >> 3, jj = e & 7, r64 = rr & 63;
+      uint32_t pk[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int s = 8 * jj + 2 * u;
+        pk[u] = pack_bf16(s <= r64 ? 1.f : 0.f, s + 1 <= r64 ? 1.f : 0.f);
+      }
+      sts128(smem + LY::L + sw128(rr, jj), make_uint4(pk[0], pk[1], pk[2], pk[3]));
+    }
+    fence_proxy_async_smem();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  if (!is_state) {
+    for (int i = threadIdx.x; i < p.R; i += NTHREADS) atomicMax(s_maxlen, stream_len(p, i));
+    __syncthreads();
+  }
+
+  if (is_state) {
+    if (warp < 8) {
+      state_warps_loop(smem, tmem, p, bars, abort_flag);
+    } else if (warp == 8) {
+      if (lane == 0) state_load_loop(smem, maps, p, bars, abort_flag);
+    } else if (warp == 9) {
+      if (lane == 0) state_mma_loop(sbase, tmem, p, bars, abort_flag);
+    }
+  } else {
+    const int g = (warp < 8) ? (warp >> 2) : ((warp - 8) & 1);
+    if (g < LY::NGROUP) {
+      Tf<TG> tf(smem, tmem, g);
+      if (warp < 8) {
+        tf.compute_loop(p, abort_flag);
+      } else if (warp < 10) {
+        tf.load_loop(maps, p, *s_maxlen, abort_flag);
+      } else if (lane == 0) {
+        tf.mma_loop(abort_flag);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0 && *abort_flag) atomicExch(p.flags + F_ABORT, 1u);
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace pipe
+}  // namespace kda

@@ -82,10 +82,10 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 
 // Warp-wide form: every lane waits, then the warp reconverges so that a
 // following .sync.aligned instruction (tcgen05.ld / st) sees all lanes.
+// The result is made warp-uniform, so a warp never splits on a timeout.
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
   const bool ok = mbar_wait(bar, parity, abort_flag);
-  __syncwarp();
-  return ok;
+  return __all_sync(0xffffffffu, ok) != 0;
 }
 
 // ------------------------------------------------------------ async proxies

@@ -88,15 +88,24 @@ typedef struct kda_shape {
 #define KDA_FLAG_VALIDATE_CU_SEQLENS 0x1u
 /* Run the tensor-core chunk path as two kernels (a fully parallel prep over
  * every (chunk, head) writing MMA-ready operands to the workspace, then the
- * inter-chunk recurrence) instead of the default single fused kernel. */
+ * inter-chunk recurrence) instead of the default pipelined kernel. */
 #define KDA_FLAG_PATH_TWO_PASS 0x2u
+/* Tuning of the pipelined tensor-core path (0 = automatic):
+ * KDA_FLAG_STATE_CTAS(n) fixes the number of state CTAs (each walks whole
+ * (sequence, head) chains), KDA_FLAG_GRID_CTAS(n) caps the number of CTAs of
+ * the launch (at most one per SM).  Values are clamped to what the problem and
+ * the device allow.  kda_chunk_fwd_workspace_size() depends on both. */
+#define KDA_FLAG_STATE_CTAS(n) ((((uint32_t)(n)) & 0xFFu) << 8)
+#define KDA_FLAG_GRID_CTAS(n) ((((uint32_t)(n)) & 0xFFu) << 16)
 
 /*
  * kda_chunk_fwd_workspace_size -- bytes of device workspace kda_chunk_fwd
- * needs for `shape`: 0 except on the two-pass tensor-core path
- * (KDA_FLAG_PATH_TWO_PASS), which needs one 82,432-byte operand slot per
- * (chunk, head).  Returns 0 for shapes the library rejects; kda_chunk_fwd
- * then reports the reason.
+ * needs for `shape` on the CURRENT device.  0 on the CUDA-core paths.  On the
+ * tensor-core path: a ring of 4 operand slots of 66,560 bytes per state CTA
+ * plus a few KB of counters (at most ~40 MB on a 148-SM B200, independent of
+ * the sequence lengths); with KDA_FLAG_PATH_TWO_PASS one 82,432-byte slot per
+ * (chunk, head).  Returns 0 for shapes the library rejects; kda_chunk_fwd then
+ * reports the reason.
  */
 size_t kda_chunk_fwd_workspace_size(const kda_shape* shape);
 
@@ -116,11 +125,17 @@ size_t kda_chunk_fwd_workspace_size(const kda_shape* shape);
  *               are ignored and on exit undefined.
  *
  * Paths: bf16 io with dk = dv = 128 and chunk = 64 runs on the tcgen05
- * tensor cores (fp32 state, bf16 operands, fp32 accumulation): by default one
- * fused kernel per call, one CTA per (sequence, head), no workspace; with
- * KDA_FLAG_PATH_TWO_PASS a prep kernel plus a recurrence kernel through the
- * workspace.  Every other supported shape, and all fp32 io, runs the fp32
- * CUDA-core recurrent kernel.  Sequences of length 0 copy S0 to S_T.
+ * tensor cores (fp32 state, bf16 operands, fp32 accumulation).  By default one
+ * cooperative launch with one CTA per SM: "state" CTAs each carry whole
+ * (sequence, head) chains through their chunks, "transform" CTAs compute the
+ * state-independent per-chunk operands in parallel and hand them over through
+ * a ring in the workspace.  q, k, v and log_alpha must then be 16-byte aligned
+ * (they are read by TMA).  With KDA_FLAG_PATH_TWO_PASS a prep kernel plus a
+ * recurrence kernel through a larger workspace.  Every other supported shape,
+ * and all fp32 io, runs the fp32 CUDA-core recurrent kernel (token by token,
+ * which keeps fp32 inputs within the 1e-4 tolerance).  Sequences of length 0
+ * copy S0 to S_T.  The call must not overlap another use of the same
+ * workspace on the GPU.
  */
 kda_status kda_chunk_fwd(const kda_shape* shape, const void* q, const void* k, const void* v,
                          const void* log_alpha, const void* beta, const float* S0,
@@ -136,25 +151,26 @@ kda_status kda_chunk_fwd(const kda_shape* shape, const void* q, const void* k, c
  * owns the GPU and offers no allocator across a C boundary, or a
  * latency-critical serving loop that bans cudaMalloc because it synchronises
  * the device and stalls every other stream.  This call takes the arguments of
- * kda_chunk_fwd without the workspace and runs the two-pass tensor-core path
- * (the one that needs scratch, KDA_FLAG_PATH_TWO_PASS) on a fixed scratch
- * array that lives in the library's device image.  (The default fused path of
- * kda_chunk_fwd needs no workspace at all.)
+ * kda_chunk_fwd without the workspace and runs the same path, with the
+ * tensor-core path's workspace (its operand ring and counters) in a fixed
+ * scratch array that lives in the library's device image.
  *
  *   - The array holds KDA_NOALLOC_SCRATCH_BYTES (64 MiB).  Every GPU that
  *     loads the library reserves it until the process exits.
  *   - A shape whose kda_chunk_fwd_workspace_size() exceeds that is rejected
- *     with KDA_ERR_WORKSPACE before anything is launched (the tensor-core
- *     path fits up to 814 (chunk, head) pairs, e.g. 16 heads x ~3,000 tokens;
- *     shapes that need no workspace have no limit).
+ *     with KDA_ERR_WORKSPACE before anything is launched.  The default
+ *     tensor-core path needs at most ~40 MB on a 148-SM B200 whatever the
+ *     sequence lengths; KDA_FLAG_PATH_TWO_PASS needs one 82,432-byte slot per
+ *     (chunk, head) and fits up to 814 of them.
  *   - Every call looks up the array's device address (cudaGetSymbolAddress)
  *     on the current device; the lookup allocates nothing.  The first call on
  *     a device may load the library's device code there, so make that first
  *     call before any stream capture begins.
  *   - Every call shares the one array, which keeps the last call's contents.
- *     The kernels write every byte of it they later read, so nothing has to be
- *     cleared between calls, but calls whose executions overlap on the GPU
- *     (different streams or host threads) race on it: serialise them.
+ *     The counters that must start at zero are cleared on the stream at the
+ *     start of every call; every other byte is written before it is read.
+ *     Calls whose executions overlap on the GPU (different streams or host
+ *     threads) race on the array: serialise them.
  *   - It allocates nothing: no cudaMalloc, cudaFree or allocating library call.
  */
 #define KDA_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)

@@ -92,10 +92,30 @@ def test_workspace_required_for_two_pass_path():
     assert call_fwd(s, ws=FAKE + 4, ws_bytes=need) == -4
 
 
-def test_fused_and_cuda_core_paths_need_no_workspace():
-    assert kda.kda_chunk_fwd_workspace_size(tc_shape()) == 0
+def test_cuda_core_paths_need_no_workspace():
     assert kda.kda_chunk_fwd_workspace_size(tc_shape(io_dtype=0)) == 0
     assert kda.kda_chunk_fwd_workspace_size(tc_shape(dk=64, dv=64)) == 0
+    assert kda.kda_chunk_fwd_workspace_size(tc_shape(chunk=32)) == 0
+
+
+def test_tuning_flags_are_accepted_and_encoded():
+    assert kda.tuning_flags(3, 10) == (3 << 8) | (10 << 16)
+    with pytest.raises(ValueError):
+        kda.tuning_flags(256, 0)
+    # the flag bits pass validation (the call then fails on the missing workspace,
+    # or on the absent device, never on the flags)
+    assert call_fwd(tc_shape(flags=kda.tuning_flags(2, 8))) in (-6, -7)
+
+
+@pytest.mark.gpu
+def test_pipelined_path_workspace_is_bounded_by_the_sm_count():
+    import torch
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    small = kda.kda_chunk_fwd_workspace_size(tc_shape())
+    big = kda.kda_chunk_fwd_workspace_size(tc_shape(B=1, T=1 << 20, H=64))
+    assert 0 < small <= big <= sms * 4 * 66560 + 65536
+    capped = kda.kda_chunk_fwd_workspace_size(tc_shape(H=64, flags=kda.tuning_flags(3, 0)))
+    assert capped < 4 * 4 * 66560 + 65536
 
 
 def test_packed_requires_single_batch_row():

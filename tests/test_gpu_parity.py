@@ -263,3 +263,29 @@ def test_final_state_may_alias_initial_state():
     S_io = x["S0"].clone()
     o2, _ = kda.kda_chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], S_io, S_T=S_io)
     assert torch.equal(o, o2) and torch.equal(S, S_io)
+
+
+# ---------------------------------------------------------------- pipelined-path scheduling
+@pytest.mark.parametrize("state_ctas,grid_ctas", [(1, 2), (1, 0), (2, 3), (3, 0), (0, 4), (0, 0)])
+def test_tc_state_cta_splits(state_ctas, grid_ctas):
+    """Packed sequences (one empty, ragged tails) over 3 heads, with the CTA
+    split forced: one state CTA walking every chain, a single transform CTA
+    feeding it, uneven streams.  Results must not depend on the split."""
+    lens = [130, 0, 64, 1, 257, 70]
+    x = gen.make_inputs(1, sum(lens), 3, 128, 128, seqlens=lens, seed=31)
+    xd = _dev(x)
+    o, S = kda.kda_chunk_fwd(xd["q"], xd["k"], xd["v"], xd["log_alpha"], xd["beta"], xd["S0"], xd["cu_seqlens"],
+                             state_ctas=state_ctas, grid_ctas=grid_ctas)
+    assert kda.kda_check_device_error() == 0
+    _check_fwd(x, TOL_BF16, o, S)
+
+
+def test_tc_split_choice_is_bit_identical():
+    """Every chunk is computed by the same arithmetic whichever CTA runs it."""
+    lens = [200, 77, 128]
+    xd = _dev(gen.make_inputs(1, sum(lens), 4, 128, 128, seqlens=lens, seed=32))
+    args = (xd["q"], xd["k"], xd["v"], xd["log_alpha"], xd["beta"], xd["S0"], xd["cu_seqlens"])
+    ref = kda.kda_chunk_fwd(*args)
+    for sc, gc in ((1, 2), (2, 0), (5, 7)):
+        o, S = kda.kda_chunk_fwd(*args, state_ctas=sc, grid_ctas=gc)
+        assert torch.equal(o, ref[0]) and torch.equal(S, ref[1]), (sc, gc)

@@ -4,15 +4,18 @@ Some users of this library run the prefill where they have no way to get
 device memory: a plugin inside a framework whose memory pool already owns the
 GPU and exposes no allocator across the C boundary, or a serving loop that
 bans cudaMalloc because it synchronises the whole device.  For them the
-library offers kda_chunk_fwd_noalloc, which runs the two-pass tensor-core
-chunk kernels (the path that needs scratch) with their workspace in a fixed
-64 MiB array inside the library instead of a caller-supplied buffer.
+library offers kda_chunk_fwd_noalloc, which runs the same tensor-core path as
+kda_chunk_fwd with that path's workspace (its operand ring and counters) in a
+fixed 64 MiB array inside the library instead of a caller-supplied buffer.
 
-These tests call it through the C ABI and check it against kda_chunk_fwd
-within the bf16 tolerance the other parity tests use, on two calls in a row
-with different inputs, so the second call also shows that what the first left
-in the shared array does not leak into its result.  The file is named to be
-collected last.
+These tests call it through the C ABI and check it against kda_chunk_fwd and
+against the fp64 oracle, within the bf16 tolerance the other parity tests use,
+on two calls in a row with different inputs: the second call also shows that
+what the first left in the shared array does not leak into its result.  A
+separate test runs kda_chunk_fwd with a workspace filled with NaN bytes: a
+finite, correct result shows the kernels never read a workspace byte they did
+not write in the same call, which is what makes sharing one array safe.  The
+file is named to be collected last.
 """
 import ctypes
 
@@ -21,6 +24,7 @@ import pytest
 import torch
 
 import gated_delta_rule_110_b200 as kda
+import oracle
 from gated_delta_rule_110_b200 import inputs as gen
 
 TOL_BF16 = 2e-2
@@ -46,13 +50,16 @@ def _call_noalloc_c_abi(x, o, S_T):
                                      p(x["beta"]), p(x["S0"]), p(x["cu_seqlens"]), p(o), p(S_T), stream)
 
 
-@pytest.mark.gpu
-def test_noalloc_matches_workspace_entry_point_on_two_calls():
-    cases = [
+def _cases():
+    return [
         gen.make_inputs(2, 200, 3, 128, 128, seed=301),                        # batched, ragged tail
         gen.make_inputs(1, 330, 2, 128, 128, seqlens=[130, 1, 199], seed=302),  # packed sequences
     ]
-    for x in cases:
+
+
+@pytest.mark.gpu
+def test_noalloc_matches_workspace_entry_point_and_oracle_on_two_calls():
+    for x in _cases():
         xd = {k: (v.cuda() if v is not None else None) for k, v in x.items()}
         o_ref, S_ref = kda.kda_chunk_fwd(xd["q"], xd["k"], xd["v"], xd["log_alpha"], xd["beta"], xd["S0"],
                                          xd["cu_seqlens"])
@@ -63,16 +70,41 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls():
         assert kda.kda_check_device_error() == 0
         assert _rel_slices(o.float().cpu(), o_ref.float().cpu(), (0, 2)) <= TOL_BF16
         assert _rel_slices(S_T.cpu(), S_ref.cpu(), (0, 1)) <= TOL_BF16
+        cu = None if x["cu_seqlens"] is None else x["cu_seqlens"].numpy()
+        o_or, S_or = oracle.forward(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["S0"], cu_seqlens=cu)
+        o_h = o.float().cpu().numpy()
+        if cu is None:
+            assert _rel_slices(o_h, o_or, (0, 2)) <= TOL_BF16
+        else:
+            for n in range(len(cu) - 1):
+                a, b = int(cu[n]), int(cu[n + 1])
+                assert _rel_slices(o_h[:, a:b], o_or[:, a:b], (0, 2)) <= TOL_BF16
+        assert _rel_slices(S_T.cpu().numpy(), S_or, (0, 1)) <= TOL_BF16
+
+
+@pytest.mark.gpu
+def test_workspace_bytes_are_written_before_they_are_read():
+    x = _cases()[1]
+    xd = {k: (v.cuda() if v is not None else None) for k, v in x.items()}
+    shape = kda.make_shape(1, xd["q"].shape[1], 2, 128, 128, 64, 3, kda.KDA_BF16, kda.KDA_BF16)
+    ws = torch.full((kda.kda_chunk_fwd_workspace_size(shape),), 0xFF, dtype=torch.uint8, device="cuda")
+    o, S = kda.kda_chunk_fwd(xd["q"], xd["k"], xd["v"], xd["log_alpha"], xd["beta"], xd["S0"], xd["cu_seqlens"],
+                             workspace=ws)
+    assert kda.kda_check_device_error() == 0
+    assert torch.isfinite(o.float()).all() and torch.isfinite(S).all()
+    o_or, S_or = oracle.forward(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["S0"],
+                                cu_seqlens=x["cu_seqlens"].numpy())
+    assert _rel_slices(S.cpu().numpy(), S_or, (0, 1)) <= TOL_BF16
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch():
     """A request larger than the built-in 64 MiB is refused before any launch
-    (host-side check, runs without a GPU)."""
+    (host-side check, runs without a GPU): the two-pass path's workspace grows
+    with the number of (chunk, head) pairs."""
     lib = kda.load_library()
-    shape = kda.make_shape(1, 65536, 16, 128, 128, 64, 0, kda.KDA_BF16, kda.KDA_BF16)
-    two_pass = kda.make_shape(1, 65536, 16, 128, 128, 64, 0, kda.KDA_BF16, kda.KDA_BF16,
-                              kda.KDA_FLAG_PATH_TWO_PASS)
-    assert kda.kda_chunk_fwd_workspace_size(two_pass) > 64 * 1024 * 1024
+    shape = kda.make_shape(1, 65536, 16, 128, 128, 64, 0, kda.KDA_BF16, kda.KDA_BF16,
+                           kda.KDA_FLAG_PATH_TWO_PASS)
+    assert kda.kda_chunk_fwd_workspace_size(shape) > 64 * 1024 * 1024
     fake = ctypes.c_void_p(0x10000)
     rc = lib.kda_chunk_fwd_noalloc(ctypes.byref(shape), fake, fake, fake, fake, fake, None, None, fake, None,
                                    None)
