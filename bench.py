@@ -393,6 +393,40 @@ def run_ours(args):
     return 0
 
 
+def run_profile(args):
+    """One leg alone, for profilers: --profile NAME runs W + K calls of that
+    workload's entry point and prints the CUDA-event time per call (no JSON)."""
+    import gated_delta_rule_110_b200 as kda
+    from gated_delta_rule_110_b200 import inputs as gen
+    torch.cuda.set_device(0)
+    kda.load_library()
+    stream = torch.cuda.current_stream()
+    w = gen.workload(args.profile)
+    if args.profile == "decode":
+        S = gen.decode_state(w.B, w.H, w.dk, w.dv, device="cuda", seed=w.seed)
+        xs = gen.decode_step_inputs(w.B, w.H, w.dk, w.dv, 0, device="cuda", seed=w.seed)
+        od = torch.empty((w.B, w.H, w.dv), dtype=torch.bfloat16, device="cuda")
+
+        def fn():
+            kda.kda_decode_step(xs["q"], xs["k"], xs["v"], xs["log_alpha"], xs["beta"], S, o=od)
+    else:
+        x = gen.workload_inputs(w, device="cuda")
+        n_seqs = 0 if x["cu_seqlens"] is None else x["cu_seqlens"].numel() - 1
+        shape = kda.make_shape(w.B, w.T, w.H, w.dk, w.dv, 64, n_seqs, kda.KDA_BF16, kda.KDA_BF16)
+        ws = torch.empty(max(kda.kda_chunk_fwd_workspace_size(shape), 1), dtype=torch.uint8, device="cuda")
+        o = torch.empty_like(x["v"])
+        S_T = torch.empty_like(x["S0"])
+
+        def fn():
+            kda.kda_chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["S0"], x["cu_seqlens"], o=o,
+                              S_T=S_T, workspace=ws)
+    t = timed(fn, args.steps, args.warmup, 1, stream)
+    err = kda.kda_check_device_error()
+    print(f"{args.profile}: {t / args.steps * 1e6:.1f} us per call over {args.steps} calls, device status {err}",
+          flush=True)
+    return 0 if err == 0 else 1
+
+
 def progress(msg: str):
     print(f"[bench] {msg}", file=sys.stderr, flush=True)
 
@@ -406,9 +440,13 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=1000)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", choices=("prefill", "varlen", "long", "decode"), default=None,
+                    help="time one workload's entry point alone (for ncu); prints no JSON line")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.profile:
+        return run_profile(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

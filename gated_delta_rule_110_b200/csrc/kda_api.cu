@@ -311,7 +311,8 @@ kda_status kda_chunk_fwd(const kda_shape* sp, const void* q, const void* k, cons
   if (N == 0) return KDA_OK;
 
   if (use_tc(s) && !use_two_pass(s) && Ttot > 0) {
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(log_alpha)) return KDA_ERR_ALIGN;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(log_alpha) || !aligned16(o))
+      return KDA_ERR_ALIGN;
     if (s.gate_dtype == KDA_BF16)
       return launch_prefill<__nv_bfloat16>(s, N, Ttot, q, k, v, log_alpha, beta, S0, cu_seqlens, o, S_T, workspace,
                                            workspace_bytes, st);

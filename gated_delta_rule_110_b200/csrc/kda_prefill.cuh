@@ -51,7 +51,7 @@ namespace pipe {
 constexpr int C = 64;
 constexpr int D = 128;
 constexpr int NTHREADS = 384;
-constexpr int NRING = 4;
+constexpr int NRING = 8;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kSpan2 = 230.0f;  // largest chunk decay of the factorised path, log2 units
 
@@ -77,12 +77,13 @@ constexpr uint32_t ST_SLOT = 0;                   // 2 ring slots
 constexpr uint32_t ST_V = 2 * SLOT;               // 2 x V tile [r][v] (two 64-value atoms)
 constexpr uint32_t ST_S = ST_V + 2 * 16384;       // S'^T [v][c] bf16, two 64-channel atoms
 constexpr uint32_t ST_U = ST_S + 32768;           // U^T [v][r] bf16
-constexpr uint32_t ST_BAR = ST_U + 16384;
+constexpr uint32_t ST_OX = ST_U + 16384;          // per-warp 16 x 128 B transpose scratch for O (8 x 2 KB)
+constexpr uint32_t ST_BAR = ST_OX + 16384;
 constexpr uint32_t ST_BYTES = ST_BAR + 256;
 // TMEM columns
-constexpr uint32_t TS_U = 0;     // U^T fp32        64
-constexpr uint32_t TS_DS = 128;  // dS^T fp32      128
-constexpr uint32_t TS_O = 256;   // 2 x O^T fp32    2 x 64
+constexpr uint32_t TS_U = 0;     // U^T fp32                       64
+constexpr uint32_t TS_DS = 128;  // dS^T fp32                     128
+constexpr uint32_t TS_O = 256;   // 2 x O [r][v] fp32 (M = 64)   2 x 128
 
 // ---- transform CTA shared memory ------------------------------------------------
 template <typename TG>
@@ -116,7 +117,10 @@ constexpr uint32_t TT_W = 192;  // W'^T fp32                        64
 // meta words
 enum { MT_DONE = 0, MT_SLOW, MT_N, MT_H, MT_J, MT_L, MT_I, MT_POS, MT_T0LO, MT_T0HI };
 // transform mbarriers
-enum { BT_RAW_FULL = 0, BT_RAW_FREE, BT_CS_GO, BT_CS_FULL, BT_AP_GO, BT_AP_FULL, BT_W_GO, BT_W_FULL, BT_FIN };
+enum {
+  BT_RAW_FULL = 0, BT_RAW_FREE, BT_CS_GO, BT_CS_FULL, BT_AP_GO, BT_AP_FULL, BT_W_GO, BT_W_FULL, BT_FIN,
+  BT_WT_STAGED, BT_WT_READ
+};
 // state mbarriers
 enum {
   BS_SLOT_FULL = 0, BS_SLOT_FREE = 2, BS_S_READY = 4, BS_U_FULL, BS_U_READY, BS_DS_FULL, BS_O_FULL,
@@ -234,12 +238,17 @@ struct Tf {
   __device__ float* betas() const { return reinterpret_cast<float*>(misc + LY::M_BETA); }
   __device__ float* gls() const { return reinterpret_cast<float*>(misc + LY::M_GL); }
   __device__ float* scs() const { return reinterpret_cast<float*>(misc + LY::M_SC); }
-  // T (fp32, [64][64]) lives in the Qa rows of the [Ka; Qa] tile once A/P is done
+  // T (fp32, [64][64]) lives in the Qa rows of the [Ka; Qa] tile once A/P is
+  // done; its 4-float groups are XOR-permuted per row like A's (tcol()).
   __device__ float* trow(int r) const {
     return reinterpret_cast<float*>(gb + LY::G_KQ + (r < 32 ? 8192 : 24576) + (r & 31) * 256);
   }
+  __device__ static int tcol(int r, int s) { return s ^ ((((r & 7) ^ ((r >> 3) & 7))) << 2); }
   __device__ float* amat() const { return reinterpret_cast<float*>(gb + LY::G_KB); }
   __device__ void bar() const { named_bar(1 + g, 128); }
+  // The cumsum operand is the raw TMA tile unless rows past the chunk end must
+  // be zeroed or fp32 gates must be split into bf16 parts first.
+  __device__ static bool needs_prep(int L) { return sizeof(TG) != 2 || L < C; }
 
   // ------------------------------------------------------------ load warp
   __device__ void load_loop(const Maps& maps, const Params& p, int maxlen, volatile int* abort_flag) {
@@ -247,6 +256,30 @@ struct Tf {
     uint32_t* gflags = p.flags;
     const long long total = static_cast<long long>(p.R) * maxlen;
     int it = 0;
+    int prev_si = -1, prev_pos = 0;  // chunk whose -W'^T copy and publication are still due (lane 0)
+    int nfinished = 0;
+    // Ships the previous chunk's -W'^T tile once the compute warps staged it,
+    // waits for every copy of that chunk to land, and publishes its ring slot.
+    auto finish_prev = [&]() -> bool {
+      if (prev_si < 0) return true;
+      const int k = nfinished;
+      if (!mbar_wait(&bars[BT_WT_STAGED], k & 1, abort_flag)) return false;
+      uint8_t* pslot = p.ring + (static_cast<size_t>(prev_si) * NRING + (prev_pos % NRING)) * SLOT;
+      bulk_s2g(pslot + R_WT, gb + LY::G_KB, 16384);
+      bulk_commit();
+      bulk_wait_read<0>();
+      mbar_arrive(&bars[BT_WT_READ]);
+      bulk_wait_all();
+      if (!*abort_flag) {
+        fence_proxy_async_global();
+        __threadfence();
+        st_release_gpu(gflags + F_REC0 + prev_si * F_REC_STRIDE + (prev_pos % NRING),
+                       static_cast<uint32_t>(prev_pos + 1));
+      }
+      ++nfinished;
+      prev_si = -1;
+      return true;
+    };
     for (;; ++it) {
       // lane 0 decides; every lane takes the same branch
       int stop = 0, done = 0, i = 0, pos = 0, n = 0, h = 0, j = 0, L = 0;
@@ -321,8 +354,14 @@ struct Tf {
           for (int qq = 0; qq < 4; ++qq)
             tma_load_2d(gb + LY::G_RL + qq * 8192, &maps.la, h * D + 32 * qq, y, &bars[BT_RAW_FULL]);
         }
+        // while this chunk's tiles are in flight, finish the previous chunk
+        if (!finish_prev()) stop = 1;
+        prev_si = i;
+        prev_pos = pos;
       }
+      if (__shfl_sync(0xffffffffu, stop, 0)) break;
     }
+    if (lane == 0 && !*abort_flag) finish_prev();
     // a load issued for an item that was never consumed must land before exit
     if (lane == 0 && it >= 1) {
       const long long t0 = clock64();
@@ -337,9 +376,14 @@ struct Tf {
     constexpr uint32_t id_ap = make_idesc_bf16(128, 64);
     constexpr uint32_t id_w = make_idesc_bf16(128, 64) | IDESC_A_MN;
     const uint32_t Lb = sbase + LY::L;
+    int nprep = 0;  // chunks whose cumsum operand the compute warps prepared first
     for (int it = 0;; ++it) {
-      if (!mbar_wait(&bars[BT_CS_GO], it & 1, abort_flag)) break;
+      if (!mbar_wait(&bars[BT_RAW_FULL], it & 1, abort_flag)) break;
       if (*reinterpret_cast<volatile int*>(&meta[MT_DONE])) break;
+      if (needs_prep(meta[MT_L])) {
+        if (!mbar_wait(&bars[BT_CS_GO], nprep & 1, abort_flag)) break;
+        ++nprep;
+      }
       tc_fence_after();
       if (sizeof(TG) == 2) {
 #pragma unroll
@@ -399,14 +443,17 @@ struct Tf {
       // the abort flag, and every barrier is still reached.
       const bool got = mbar_wait_warp(&bars[BT_RAW_FULL], it & 1, abort_flag);
       const bool fin = got && *reinterpret_cast<volatile int*>(&meta[MT_DONE]) != 0;
-      if (named_bar_or(1 + g, 128, !got || fin || *abort_flag)) {
-        if (gt == 0 && fin && !*abort_flag) mbar_arrive(&bars[BT_CS_GO]);
-        break;
-      }
+      if (named_bar_or(1 + g, 128, !got || fin || *abort_flag)) break;
       const int L = meta[MT_L];
       const int si = meta[MT_I];
       const int pos = meta[MT_POS];
       const int hh = meta[MT_H];
+      if (gt == 0) {
+        // this chunk's ring slot must have been copied out by its state CTA
+        if (pos + 1 - NRING > 0)
+          spin_geq(gflags + F_REC0 + si * F_REC_STRIDE + F_CONSUMED, static_cast<uint32_t>(pos + 1 - NRING),
+                   gflags + F_ABORT, abort_flag);
+      }
       const int64_t t0 = static_cast<int64_t>((static_cast<uint64_t>(static_cast<uint32_t>(meta[MT_T0HI])) << 32) |
                                               static_cast<uint32_t>(meta[MT_T0LO]));
       uint8_t* slot = p.ring + (static_cast<size_t>(si) * NRING + (pos % NRING)) * SLOT;
@@ -415,8 +462,13 @@ struct Tf {
       // chunk as soon as the raw tiles are released)
       const float beta_r = gt < L ? ld_gate(static_cast<const TG*>(p.beta) + (t0 + gt) * p.H + hh) : 0.f;
 
-      // ---- C1: prepare the cumsum operand -------------------------------------
-      if (sizeof(TG) == 2) {
+      // the previous chunk's -W'^T staging (KB area) must have been read before
+      // anything here writes that area
+      if (it >= 1) mbar_wait_warp(&bars[BT_WT_READ], (it - 1) & 1, abort_flag);
+
+      // ---- C1: prepare the cumsum operand (when the raw tile is not usable) ----
+      if (!needs_prep(L)) {
+      } else if (sizeof(TG) == 2) {
         if (L < C) {
           for (int e = gt; e < (C - L) * 16; e += 128) {
             const int rr = L + (e >> 4), hf = (e >> 3) & 1, jj = e & 7;
@@ -456,9 +508,11 @@ struct Tf {
           }
         }
       }
-      fence_proxy_async_smem();
-      bar();
-      if (gt == 0) mbar_arrive(&bars[BT_CS_GO]);
+      if (needs_prep(L)) {
+        fence_proxy_async_smem();
+        bar();
+        if (gt == 0) mbar_arrive(&bars[BT_CS_GO]);
+      }
 
       // ---- C2: cumulative decay -> scaled tiles ---------------------------------
       if (gt < C) sbeta[gt] = beta_r;  // published by the barriers below
@@ -484,10 +538,6 @@ struct Tf {
           steep = steep || (-g2[u] > kSpan2);
         }
       }
-      // the ring slot must have been copied out by its state CTA
-      if (gt == 0 && pos + 1 - NRING > 0)
-        spin_geq(gflags + F_REC0 + si * F_REC_STRIDE + F_CONSUMED, static_cast<uint32_t>(pos + 1 - NRING),
-                 gflags + F_ABORT, abort_flag);
       const bool slow = named_bar_or(1 + g, 128, steep);
       {
         // per channel: sc = 2^{g_last/2} (1 on the exact path), gamma_C = 2^{g_last}
@@ -503,6 +553,13 @@ struct Tf {
 #pragma unroll
         for (int jj = 0; jj < 8; ++jj) {
           const int c0 = 64 * ch + 8 * jj;
+          const float4 gla = *reinterpret_cast<const float4*>(sgl + c0);
+          const float4 glb = *reinterpret_cast<const float4*>(sgl + c0 + 4);
+          const float4 sca = *reinterpret_cast<const float4*>(ssc + c0);
+          const float4 scb = *reinterpret_cast<const float4*>(ssc + c0 + 4);
+          const float rf8[8] = {0.5f * gla.x, 0.5f * gla.y, 0.5f * gla.z, 0.5f * gla.w,
+                                0.5f * glb.x, 0.5f * glb.y, 0.5f * glb.z, 0.5f * glb.w};
+          const float sc8[8] = {sca.x, sca.y, sca.z, sca.w, scb.x, scb.y, scb.z, scb.w};
           uint4 kw = lds128(gb + LY::G_RK + ch * 8192 + sw128(r, jj));
           uint4 qw = lds128(gb + LY::G_RQ + ch * 8192 + sw128(r, jj));
           if (r >= L) kw = qw = make_uint4(0u, 0u, 0u, 0u);
@@ -512,7 +569,7 @@ struct Tf {
           for (int u = 0; u < 4; ++u) {
             const int c = c0 + 2 * u;
             const float2 kx = bf2f(kk4[u]), qx = bf2f(qq4[u]);
-            const float rf0 = 0.5f * sgl[c], rf1 = 0.5f * sgl[c + 1];
+            const float rf0 = rf8[2 * u], rf1 = rf8[2 * u + 1];
             const float x0 = g2[8 * jj + 2 * u], x1 = g2[8 * jj + 2 * u + 1];
             const float e10 = ex2_approx(x0 - rf0), e11 = ex2_approx(x1 - rf1);
             const float e20 = ex2_approx(rf0 - x0), e21 = ex2_approx(rf1 - x1);
@@ -520,14 +577,13 @@ struct Tf {
             qa[u] = pack_bf16(qx.x * e10, qx.y * e11);
             const float b0 = kx.x * e20, b1 = kx.y * e21;
             kb[u] = pack_bf16(b0, b1);
-            kt[u] = pack_bf16(b0 * ssc[c], b1 * ssc[c + 1]);
+            kt[u] = pack_bf16(b0 * sc8[2 * u], b1 * sc8[2 * u + 1]);
           }
-          const uint4 kav = make_uint4(ka[0], ka[1], ka[2], ka[3]), qav = make_uint4(qa[0], qa[1], qa[2], qa[3]);
-          sts128(gb + LY::G_KQ + ch * 16384 + sw128(r, jj), kav);
-          sts128(gb + LY::G_KQ + ch * 16384 + sw128(64 + r, jj), qav);
+          sts128(gb + LY::G_KQ + ch * 16384 + sw128(r, jj), make_uint4(ka[0], ka[1], ka[2], ka[3]));
+          sts128(gb + LY::G_KQ + ch * 16384 + sw128(64 + r, jj), make_uint4(qa[0], qa[1], qa[2], qa[3]));
           sts128(gb + LY::G_KB + ch * 8192 + sw128(r, jj), make_uint4(kb[0], kb[1], kb[2], kb[3]));
-          stg128(slot + R_QA + ch * 8192 + sw128(r, jj), qav);
-          stg128(slot + R_KT + ch * 8192 + sw128(r, jj), make_uint4(kt[0], kt[1], kt[2], kt[3]));
+          // Kt replaces the raw k chunk this thread just read (ring layout)
+          sts128(gb + LY::G_RK + ch * 8192 + sw128(r, jj), make_uint4(kt[0], kt[1], kt[2], kt[3]));
         }
       } else {
         // ---- exact path: A and P term by term from g (fp32, in the KQ area) ------
@@ -558,7 +614,8 @@ struct Tf {
             }
           }
           Af[swzA(ar, as)] = as < ar ? sbeta[ar] * a : 0.f;
-          *reinterpret_cast<__nv_bfloat16*>(slot + R_PP + sw128(ar, as >> 3) + (as & 7) * 2) = __float2bfloat16_rn(pp);
+          *reinterpret_cast<__nv_bfloat16*>(gb + LY::G_RL + sw128(ar, as >> 3) + (as & 7) * 2) =
+              __float2bfloat16_rn(pp);
         }
         bar();  // g is dead; Ka / Qa overwrite it
 #pragma unroll
@@ -580,11 +637,9 @@ struct Tf {
             qa[u] = pack_bf16(qx.x * gm0, qx.y * gm1);
             kt[u] = pack_bf16(kx.x * ps0, kx.y * ps1);
           }
-          const uint4 kav = make_uint4(ka[0], ka[1], ka[2], ka[3]), qav = make_uint4(qa[0], qa[1], qa[2], qa[3]);
-          sts128(gb + LY::G_KQ + ch * 16384 + sw128(r, jj), kav);
-          sts128(gb + LY::G_KQ + ch * 16384 + sw128(64 + r, jj), qav);
-          stg128(slot + R_QA + ch * 8192 + sw128(r, jj), qav);
-          stg128(slot + R_KT + ch * 8192 + sw128(r, jj), make_uint4(kt[0], kt[1], kt[2], kt[3]));
+          sts128(gb + LY::G_KQ + ch * 16384 + sw128(r, jj), make_uint4(ka[0], ka[1], ka[2], ka[3]));
+          sts128(gb + LY::G_KQ + ch * 16384 + sw128(64 + r, jj), make_uint4(qa[0], qa[1], qa[2], qa[3]));
+          sts128(gb + LY::G_RK + ch * 8192 + sw128(r, jj), make_uint4(kt[0], kt[1], kt[2], kt[3]));
         }
       }
       fence_proxy_async_smem();
@@ -592,8 +647,12 @@ struct Tf {
       bar();
       if (gt == 0) {
         meta[MT_SLOW] = slow ? 1 : 0;
-        mbar_arrive(&bars[BT_RAW_FREE]);
         mbar_arrive(&bars[BT_AP_GO]);
+        // Qa (the lower half of each [Ka; Qa] atom) and Kt go to the ring slot
+        bulk_s2g(slot + R_QA, gb + LY::G_KQ + 8192, 8192);
+        bulk_s2g(slot + R_QA + 8192, gb + LY::G_KQ + 16384 + 8192, 8192);
+        bulk_s2g(slot + R_KT, gb + LY::G_RK, 16384);
+        bulk_commit();
       }
 
       // ---- C3: A / P epilogue -------------------------------------------------------
@@ -635,38 +694,55 @@ struct Tf {
               const int s0 = 8 * jj + 2 * u;
               pk[u] = pack_bf16(s0 <= rp ? x[s0] : 0.f, s0 + 1 <= rp ? x[s0 + 1] : 0.f);
             }
-            stg128(slot + R_PP + sw128(rp, jj), make_uint4(pk[0], pk[1], pk[2], pk[3]));
+            sts128(gb + LY::G_RL + sw128(rp, jj), make_uint4(pk[0], pk[1], pk[2], pk[3]));
           }
         }
+      }
+      fence_proxy_async_smem();
+      bar();
+      if (gt == 0) {
+        bulk_s2g(slot + R_PP, gb + LY::G_RL, 8192);
+        bulk_commit();
+        // the inverse writes T over Qa: every copy out of shared memory must
+        // have read its source; then the raw tiles are free for the next chunk
+        bulk_wait_read<0>();
+        mbar_arrive(&bars[BT_RAW_FREE]);
       }
       bar();
 
       // ---- C4: T = (I + A)^-1, blocked forward substitution (fp32) ---------------
       invert(sbeta);
-      // Tb = T Diag(beta) -> bf16 [r][s] (local MMA operand and ring slot)
+      // Tb = T Diag(beta) -> bf16 [r][s] (local MMA operand, shipped to the ring
+      // slot); 8 threads share a row, one 16-byte chunk of 8 columns each
       {
-        const int tr = gt >> 1, sh = gt & 1;
-        const float* Tr = trow(tr);
+        const int jq = gt & 7;
+        const int s0 = 8 * jq;
+        const float4 b0 = *reinterpret_cast<const float4*>(sbeta + s0);
+        const float4 b1 = *reinterpret_cast<const float4*>(sbeta + s0 + 4);
 #pragma unroll
-        for (int j4 = 0; j4 < 4; ++j4) {
-          const int s0 = 32 * sh + 8 * j4;
-          uint32_t pk[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int s = s0 + 2 * u;
-            const float a = (s >> 4) <= (tr >> 4) ? Tr[s] * sbeta[s] : 0.f;
-            const float b = ((s + 1) >> 4) <= (tr >> 4) ? Tr[s + 1] * sbeta[s + 1] : 0.f;
-            pk[u] = pack_bf16(a, b);
+        for (int pass = 0; pass < 4; ++pass) {
+          const int tr = 16 * pass + (gt >> 3);
+          uint32_t pk[4] = {0u, 0u, 0u, 0u};
+          if ((s0 >> 4) <= (tr >> 4)) {
+            const float* Tr = trow(tr);
+            const float4 t0 = *reinterpret_cast<const float4*>(Tr + tcol(tr, s0));
+            const float4 t1 = *reinterpret_cast<const float4*>(Tr + tcol(tr, s0 + 4));
+            pk[0] = pack_bf16(t0.x * b0.x, t0.y * b0.y);
+            pk[1] = pack_bf16(t0.z * b0.z, t0.w * b0.w);
+            pk[2] = pack_bf16(t1.x * b1.x, t1.y * b1.y);
+            pk[3] = pack_bf16(t1.z * b1.z, t1.w * b1.w);
           }
-          const uint4 w = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          sts128(gb + LY::G_TB + sw128(tr, s0 >> 3), w);
-          stg128(slot + R_TB + sw128(tr, s0 >> 3), w);
+          sts128(gb + LY::G_TB + sw128(tr, jq), make_uint4(pk[0], pk[1], pk[2], pk[3]));
         }
       }
       fence_proxy_async_smem();
       tc_fence_before();
       bar();
-      if (gt == 0) mbar_arrive(&bars[BT_W_GO]);
+      if (gt == 0) {
+        mbar_arrive(&bars[BT_W_GO]);
+        bulk_s2g(slot + R_TB, gb + LY::G_TB, 8192);
+        bulk_commit();
+      }
 
       // ---- C5: -W'^T -> ring slot, then publish --------------------------------------
       mbar_wait_warp(&bars[BT_W_FULL], it & 1, abort_flag);
@@ -683,75 +759,140 @@ struct Tf {
             uint32_t pk[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) pk[u] = pack_bf16(-x[8 * j4 + 2 * u], -x[8 * j4 + 2 * u + 1]);
-            stg128(slot + R_WT + sw128(c, 4 * hf + j4), make_uint4(pk[0], pk[1], pk[2], pk[3]));
+            sts128(gb + LY::G_KB + sw128(c, 4 * hf + j4), make_uint4(pk[0], pk[1], pk[2], pk[3]));
           }
         }
       }
+      fence_proxy_async_smem();
       tc_fence_before();
       bar();
-      if (gt == 0 && !*abort_flag) {
-        __threadfence();
-        st_release_gpu(gflags + F_REC0 + si * F_REC_STRIDE + (pos % NRING), static_cast<uint32_t>(pos + 1));
+      if (gt == 0) {
+        // this thread's copies (Qa, Kt, P, Tb) have landed; the load warp ships
+        // -W'^T and publishes the slot
+        bulk_wait_all();
+        fence_proxy_async_global();
+        mbar_arrive(&bars[BT_WT_STAGED]);
       }
     }
   }
 
   // T = (I + A)^-1 for the strictly lower-triangular A (fp32, swizzled rows in
-  // the KB area), written to trow().  Diagonal 16 x 16 blocks by column-wise
+  // the KB area), written to trow().  Diagonal 16 x 16 blocks by row-wise
   // forward substitution; then block levels d = 1, 2, 3:
   //   T_IJ = -T_II sum_{K=J}^{I-1} A_IK T_KJ      (I - J = d)
+  // Block indices are compile-time, so every shared-memory offset except the
+  // thread's own row / column is an immediate.
+  __device__ static int swz4(int r) { return (((r & 7) ^ ((r >> 3) & 7))) << 2; }
+
+  // X_b[i][j0, j0+1] = sum_{K=J}^{I-1} A_IK[i][:] T_KJ[:][j0, j0+1]
+  template <int I, int J>
+  __device__ __forceinline__ void level_x(float* X, int b, int i, int j0) const {
+    const float* Ar = amat() + (16 * I + i) * 64;
+    const int sa = swz4(16 * I + i);
+    float a0 = 0.f, a1 = 0.f, c0 = 0.f, c1 = 0.f;
+#pragma unroll
+    for (int K = J; K < I; ++K) {
+#pragma unroll
+      for (int g4 = 0; g4 < 4; ++g4) {
+        const float4 av = *reinterpret_cast<const float4*>(Ar + ((16 * K + 4 * g4) ^ sa));
+        const float aa[4] = {av.x, av.y, av.z, av.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int rt = 16 * K + 4 * g4 + u;
+          const float2 tv = *reinterpret_cast<const float2*>(trow(rt) + tcol(rt, 16 * J + j0));
+          if (u & 1) {
+            c0 += aa[u] * tv.x;
+            c1 += aa[u] * tv.y;
+          } else {
+            a0 += aa[u] * tv.x;
+            a1 += aa[u] * tv.y;
+          }
+        }
+      }
+    }
+    *reinterpret_cast<float2*>(X + (b * 16 + i) * 16 + j0) = make_float2(a0 + c0, a1 + c1);
+  }
+  // T_IJ[i][j0, j0+1] = -T_II[i][:] X_b[:][j0, j0+1]
+  template <int I, int J>
+  __device__ __forceinline__ void level_t(const float* X, int b, int i, int j0) {
+    const int rt = 16 * I + i;
+    float* Tr = trow(rt);
+    const int st = swz4(rt);
+    float a0 = 0.f, a1 = 0.f, c0 = 0.f, c1 = 0.f;
+#pragma unroll
+    for (int g4 = 0; g4 < 4; ++g4) {
+      const float4 tv = *reinterpret_cast<const float4*>(Tr + ((16 * I + 4 * g4) ^ st));
+      const float tt[4] = {tv.x, tv.y, tv.z, tv.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float2 xv = *reinterpret_cast<const float2*>(X + (b * 16 + 4 * g4 + u) * 16 + j0);
+        if (u & 1) {
+          c0 += tt[u] * xv.x;
+          c1 += tt[u] * xv.y;
+        } else {
+          a0 += tt[u] * xv.x;
+          a1 += tt[u] * xv.y;
+        }
+      }
+    }
+    *reinterpret_cast<float2*>(Tr + ((16 * J + j0) ^ st)) = make_float2(-(a0 + c0), -(a1 + c1));
+  }
+
   __device__ void invert(const float* sbeta) {
     const int gt = threadIdx.x - 128 * g;
     const float* Af = amat();
     float* X = reinterpret_cast<float*>(gb + LY::G_TB);  // scratch, [3][16][16]
     if (gt < 64) {
+      // column jc of T_II: x_i = delta_ij - sum_{m<i} A_II[i][m] x_m, one row at a time
       const int I = gt >> 4, jc = gt & 15;
       float x[16];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) x[i] = i == jc ? 1.f : 0.f;
+      for (int ii = 0; ii < 16; ++ii) {
+        const int ra = 16 * I + ii;
+        const float* Ar = Af + ra * 64;
+        const int sa = swz4(ra);
+        float acc0 = ii == jc ? 1.f : 0.f, acc1 = 0.f;
 #pragma unroll
-      for (int m = 0; m < 15; ++m) {
-        const float xm = x[m];
+        for (int g4 = 0; g4 < 4; ++g4) {
+          if (4 * g4 < ii) {
+            const float4 av = *reinterpret_cast<const float4*>(Ar + ((16 * I + 4 * g4) ^ sa));
+            const float aa[4] = {av.x, av.y, av.z, av.w};
 #pragma unroll
-        for (int i = m + 1; i < 16; ++i) x[i] -= Af[swzA(16 * I + i, 16 * I + m)] * xm;
-      }
-#pragma unroll
-      for (int i = 0; i < 16; ++i) trow(16 * I + i)[16 * I + jc] = x[i];
-    }
-    bar();
-    const int i = gt >> 3, j = 2 * (gt & 7);  // each thread: row i, columns j, j+1 of a 16 x 16 block
-    for (int d = 1; d < 4; ++d) {
-      const int nb = 4 - d;
-      for (int b = 0; b < nb; ++b) {
-        const int I = b + d, J = b;
-        float a0 = 0.f, a1 = 0.f;
-        for (int K = J; K < I; ++K) {
-#pragma unroll
-          for (int m = 0; m < 16; ++m) {
-            const float av = Af[swzA(16 * I + i, 16 * K + m)];
-            const float2 tv = *reinterpret_cast<const float2*>(trow(16 * K + m) + 16 * J + j);
-            a0 += av * tv.x;
-            a1 += av * tv.y;
+            for (int u = 0; u < 4; ++u) {
+              if (4 * g4 + u < ii) {
+                if (u & 1)
+                  acc1 -= aa[u] * x[4 * g4 + u];
+                else
+                  acc0 -= aa[u] * x[4 * g4 + u];
+              }
+            }
           }
         }
-        *reinterpret_cast<float2*>(X + (b * 16 + i) * 16 + j) = make_float2(a0, a1);
+        x[ii] = acc0 + acc1;
       }
-      bar();
-      for (int b = 0; b < nb; ++b) {
-        const int I = b + d, J = b;
-        float a0 = 0.f, a1 = 0.f;
-        const float* Ti = trow(16 * I + i);
 #pragma unroll
-        for (int m = 0; m < 16; ++m) {
-          const float tv = Ti[16 * I + m];
-          const float2 xv = *reinterpret_cast<const float2*>(X + (b * 16 + m) * 16 + j);
-          a0 += tv * xv.x;
-          a1 += tv * xv.y;
-        }
-        *reinterpret_cast<float2*>(trow(16 * I + i) + 16 * J + j) = make_float2(-a0, -a1);
-      }
-      bar();
+      for (int ii = 0; ii < 16; ++ii) trow(16 * I + ii)[tcol(16 * I + ii, 16 * I + jc)] = x[ii];
     }
+    bar();
+    const int i = gt >> 3, j0 = 2 * (gt & 7);  // each thread: row i, columns j0, j0+1 of a 16 x 16 block
+    level_x<1, 0>(X, 0, i, j0);
+    level_x<2, 1>(X, 1, i, j0);
+    level_x<3, 2>(X, 2, i, j0);
+    bar();
+    level_t<1, 0>(X, 0, i, j0);
+    level_t<2, 1>(X, 1, i, j0);
+    level_t<3, 2>(X, 2, i, j0);
+    bar();
+    level_x<2, 0>(X, 0, i, j0);
+    level_x<3, 1>(X, 1, i, j0);
+    bar();
+    level_t<2, 0>(X, 0, i, j0);
+    level_t<3, 1>(X, 1, i, j0);
+    bar();
+    level_x<3, 0>(X, 0, i, j0);
+    bar();
+    level_t<3, 0>(X, 0, i, j0);
+    bar();
   }
 };
 
@@ -826,7 +967,7 @@ __device__ __forceinline__ void state_mma_loop(uint32_t sbase, uint32_t tmem, co
                                                volatile int* abort_flag) {
   constexpr uint32_t id_uv = make_idesc_bf16(128, 64) | IDESC_A_MN;
   constexpr uint32_t id_us = make_idesc_bf16(128, 64) | IDESC_B_MN;
-  constexpr uint32_t id_n64 = make_idesc_bf16(128, 64);
+  constexpr uint32_t id_o = make_idesc_bf16(64, 128);
   constexpr uint32_t id_ds = make_idesc_bf16(128, 128) | IDESC_B_MN;
   const int i = blockIdx.x;
   int pos = 0;
@@ -852,14 +993,15 @@ __device__ __forceinline__ void state_mma_loop(uint32_t sbase, uint32_t tmem, co
         mma_bf16_ss(tmem + TS_U, make_sdesc_sw128(sbase + ST_S + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
                     make_sdesc_sw128(slot + R_WT + kk * 2048, 8192, 1024), id_us, 1);
       mma_commit(&bars[BS_U_FULL]);
-      // O^T = S'^T Qa^T  (buffer b, free once position pos-2 was read out)
+      // O = Qa S'  (M = 64 rows r, N = 128 values v; buffer b, free once
+      // position pos-2 was read out; S' is the K-major B operand [v][c])
       if (pos >= 2 && !mbar_wait(&bars[BS_O_FREE + b], ((pos - 2) >> 1) & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk)
-        mma_bf16_ss(tmem + TS_O + 64 * b,
-                    make_sdesc_sw128(sbase + ST_S + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                    make_sdesc_sw128(slot + R_QA + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), id_n64, kk > 0);
+        mma_bf16_ss(tmem + TS_O + 128 * b,
+                    make_sdesc_sw128(slot + R_QA + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024),
+                    make_sdesc_sw128(sbase + ST_S + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024), id_o, kk > 0);
       if (!mbar_wait(&bars[BS_U_READY], pos & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
       // dS^T = U^T Kt
@@ -868,11 +1010,11 @@ __device__ __forceinline__ void state_mma_loop(uint32_t sbase, uint32_t tmem, co
         mma_bf16_ss(tmem + TS_DS, make_sdesc_sw128(sbase + ST_U + kk * 32, 16, 1024),
                     make_sdesc_sw128(slot + R_KT + kk * 2048, 8192, 1024), id_ds, kk > 0);
       mma_commit(&bars[BS_DS_FULL]);
-      // O^T += U^T P^T
+      // O += P U  (U^T [v][r] is the K-major B operand)
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        mma_bf16_ss(tmem + TS_O + 64 * b, make_sdesc_sw128(sbase + ST_U + kk * 32, 16, 1024),
-                    make_sdesc_sw128(slot + R_PP + kk * 32, 16, 1024), id_n64, 1);
+        mma_bf16_ss(tmem + TS_O + 128 * b, make_sdesc_sw128(slot + R_PP + kk * 32, 16, 1024),
+                    make_sdesc_sw128(sbase + ST_U + kk * 32, 16, 1024), id_o, 1);
       mma_commit(&bars[BS_O_FULL + b]);
       mma_commit(&bars[BS_SLOT_FREE + s]);
     }
@@ -901,21 +1043,49 @@ __device__ __forceinline__ void state_warps_loop(uint8_t* smem, uint32_t tmem, c
   int64_t prev_t0 = 0;
   bool have_prev = false;
 
+  // O of position pp -> global.  The M = 64 accumulator keeps row r in TMEM
+  // lane 32 (r / 16) + r % 16, so lanes 0-15 of each warp hold one output row
+  // each; a thread stores its 64 values (columns 64 hf ...) with 16-byte
+  // stores, rows past the sequence end skipped.
   auto o_pass = [&](int pp) -> bool {
     const int b = pp & 1;
     if (!mbar_wait_warp(&bars[BS_O_FULL + b], (pp >> 1) & 1, abort_flag)) return false;
     tc_fence_after();
-    float x[32];
-    tmem_ld32(tmem + lane_off + TS_O + 64 * b + 32 * hf, x);
-    tmem_wait_ld();
+    float x[64];
+    {
+      float t[32];
+      tmem_ld32(tmem + lane_off + TS_O + 128 * b + 64 * hf, t);
+      tmem_wait_ld();
+#pragma unroll
+      for (int u = 0; u < 32; ++u) x[u] = t[u];
+      tmem_ld32(tmem + lane_off + TS_O + 128 * b + 64 * hf + 32, t);
+      tmem_wait_ld();
+#pragma unroll
+      for (int u = 0; u < 32; ++u) x[32 + u] = t[u];
+    }
     tc_fence_before();
     mbar_arrive(&bars[BS_O_FREE + b]);
-    __nv_bfloat16* op = p.o + (prev_t0 * p.H + prev_h) * D + v;
+    // lanes 0-15 hold rows 16 q + lane; transpose through the warp's scratch
+    // (128-byte rows, 16-byte chunks XOR-swizzled by row) so that each store
+    // instruction writes 4 whole 128-byte row segments
+    uint8_t* xs = smem + ST_OX + warp * 2048;
+    if (lane < 16) {
 #pragma unroll
-    for (int u = 0; u < 32; ++u) {
-      const int rr = 32 * hf + u;
-      if (rr < prev_L) op[static_cast<int64_t>(rr) * p.H * D] = __float2bfloat16_rn(x[u]);
+      for (int c8 = 0; c8 < 8; ++c8)
+        sts128(xs + sw128(lane, c8),
+               make_uint4(pack_bf16(x[8 * c8], x[8 * c8 + 1]), pack_bf16(x[8 * c8 + 2], x[8 * c8 + 3]),
+                          pack_bf16(x[8 * c8 + 4], x[8 * c8 + 5]), pack_bf16(x[8 * c8 + 6], x[8 * c8 + 7])));
     }
+    __syncwarp();
+#pragma unroll
+    for (int k4 = 0; k4 < 4; ++k4) {
+      const int row = 4 * k4 + (lane >> 3), c8 = lane & 7;
+      const int rr = 16 * q + row;
+      const uint4 w = lds128(xs + sw128(row, c8));
+      if (rr < prev_L)
+        *reinterpret_cast<uint4*>(p.o + ((prev_t0 + rr) * p.H + prev_h) * D + 64 * hf + 8 * c8) = w;
+    }
+    __syncwarp();
     return true;
   };
 
@@ -936,22 +1106,27 @@ __device__ __forceinline__ void state_warps_loop(uint8_t* smem, uint32_t tmem, c
       if (!mbar_wait_warp(&bars[BS_SLOT_FULL + s], (pos >> 1) & 1, abort_flag)) { ok = false; break; }
       // S'^T = bf16(sc S^T) -> shared memory (A operand); S <- gamma_C S
       {
-        const float* sc = reinterpret_cast<const float*>(slot + R_VEC) + 64 * hf;
-        const float* gc = reinterpret_cast<const float*>(slot + R_VEC) + 128 + 64 * hf;
+        const float4* sc4 = reinterpret_cast<const float4*>(slot + R_VEC) + 16 * hf;
+        const float4* gc4 = reinterpret_cast<const float4*>(slot + R_VEC) + 32 + 16 * hf;
 #pragma unroll
         for (int jj = 0; jj < 8; ++jj) {
-          uint32_t pk[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int c = 8 * jj + 2 * u;
-            pk[u] = pack_bf16(S[c] * sc[c], S[c + 1] * sc[c + 1]);
-          }
-          sts128(smem + ST_S + hf * 16384 + sw128(v, jj), make_uint4(pk[0], pk[1], pk[2], pk[3]));
+          const float4 a = sc4[2 * jj], b = sc4[2 * jj + 1];
+          const int c = 8 * jj;
+          const uint4 w = make_uint4(pack_bf16(S[c] * a.x, S[c + 1] * a.y), pack_bf16(S[c + 2] * a.z, S[c + 3] * a.w),
+                                     pack_bf16(S[c + 4] * b.x, S[c + 5] * b.y),
+                                     pack_bf16(S[c + 6] * b.z, S[c + 7] * b.w));
+          sts128(smem + ST_S + hf * 16384 + sw128(v, jj), w);
         }
         fence_proxy_async_smem();
         mbar_arrive(&bars[BS_S_READY]);
 #pragma unroll
-        for (int u = 0; u < 64; ++u) S[u] *= gc[u];
+        for (int u4 = 0; u4 < 16; ++u4) {
+          const float4 gg = gc4[u4];
+          S[4 * u4] *= gg.x;
+          S[4 * u4 + 1] *= gg.y;
+          S[4 * u4 + 2] *= gg.z;
+          S[4 * u4 + 3] *= gg.w;
+        }
       }
       if (have_prev && !o_pass(pos - 1)) { ok = false; break; }
       // U^T -> bf16 shared memory (A operand)
@@ -1048,7 +1223,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     } else {
       for (int g = 0; g < LY::NGROUP; ++g) {
         uint64_t* gbars = reinterpret_cast<uint64_t*>(smem + LY::MISC + g * LY::MISC_GROUP + LY::M_BAR);
-        for (int b = 0; b <= BT_FIN; ++b) mbar_init(&gbars[b], 1);
+        for (int b = 0; b <= BT_WT_READ; ++b) mbar_init(&gbars[b], 1);
       }
     }
     fence_mbar_init();

@@ -67,7 +67,11 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
 // leaves the CTA's abort flag raised) if the CTA is aborting or the wait ran
 // out of its cycle budget.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
-  if (mbar_try_wait(bar, parity)) return true;
+  // spin briefly (short waits, e.g. an MMA round trip, resume at once), then
+  // let the hardware park the thread between checks
+#pragma unroll 1
+  for (int i = 0; i < 64; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_try_wait_sleep(bar, parity)) {
     if (*abort_flag) return false;

@@ -101,7 +101,7 @@ typedef struct kda_shape {
 /*
  * kda_chunk_fwd_workspace_size -- bytes of device workspace kda_chunk_fwd
  * needs for `shape` on the CURRENT device.  0 on the CUDA-core paths.  On the
- * tensor-core path: a ring of 4 operand slots of 66,560 bytes per state CTA
+ * tensor-core path: a ring of 8 operand slots of 66,560 bytes per state CTA
  * plus a few KB of counters (at most ~40 MB on a 148-SM B200, independent of
  * the sequence lengths); with KDA_FLAG_PATH_TWO_PASS one 82,432-byte slot per
  * (chunk, head).  Returns 0 for shapes the library rejects; kda_chunk_fwd then

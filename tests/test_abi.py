@@ -113,9 +113,9 @@ def test_pipelined_path_workspace_is_bounded_by_the_sm_count():
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     small = kda.kda_chunk_fwd_workspace_size(tc_shape())
     big = kda.kda_chunk_fwd_workspace_size(tc_shape(B=1, T=1 << 20, H=64))
-    assert 0 < small <= big <= sms * 4 * 66560 + 65536
+    assert 0 < small <= big <= sms * 8 * 66560 + 65536
     capped = kda.kda_chunk_fwd_workspace_size(tc_shape(H=64, flags=kda.tuning_flags(3, 0)))
-    assert capped < 4 * 4 * 66560 + 65536
+    assert capped < 4 * 8 * 66560 + 65536
 
 
 def test_packed_requires_single_batch_row():
