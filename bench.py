@@ -264,6 +264,96 @@ def run_reference(args):
     return 0
 
 
+PROFILE_DIR = ROOT / "profiles"
+KERNEL_SOURCES = ("gated_delta_rule_110_b200/csrc/kda_prefill.cuh", "gated_delta_rule_110_b200/csrc/kda_ptx.cuh",
+                  "gated_delta_rule_110_b200/csrc/kda_recurrent.cuh", "gated_delta_rule_110_b200/csrc/kda_api.cu")
+
+
+def kernel_sources_hash() -> str:
+    """sha256 (16 hex digits) of the kernel sources the ncu captures describe."""
+    import hashlib
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        h.update((ROOT / rel).read_bytes())
+    return h.hexdigest()[:16]
+
+
+def profiled_counters():
+    """Per-launch DRAM traffic and tensor-pipe activity recorded from ncu
+    captures in profiles/*.md (lines "counter <workload> <name> <value>"),
+    valid only while the kernel sources still hash to the value the summary
+    was taken at (line "kernel_sources_sha <hex>")."""
+    import re
+    out = {}
+    cur = kernel_sources_hash()
+    for f in sorted(PROFILE_DIR.glob("*.md")):
+        text = f.read_text()
+        m = re.search(r"^kernel_sources_sha (\w+)", text, re.M)
+        if not m or m.group(1) != cur:
+            continue
+        for wl, name, val in re.findall(r"^counter (\w+) (\w+) ([0-9.eE+-]+)", text, re.M):
+            out.setdefault(wl, {})[name] = float(val)
+    return out
+
+
+def cpu_model() -> str:
+    try:
+        for line in Path("/proc/cpuinfo").read_text().splitlines():
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def prefill_leg(kda, gen, wname, steps, warmup, world, rank, local, stream, peaks, peak_src, counters):
+    """Times kda_chunk_fwd on one workload; returns its JSON object."""
+    w = gen.workload(wname)
+    x = gen.workload_inputs(w, device="cuda", seed_offset=rank)
+    cu = x["cu_seqlens"]
+    n_seqs = 0 if cu is None else cu.numel() - 1
+    N = w.B if cu is None else n_seqs
+    shape = kda.make_shape(w.B, w.T, w.H, w.dk, w.dv, 64, n_seqs, kda.KDA_BF16, kda.KDA_BF16)
+    ws = torch.empty(max(kda.kda_chunk_fwd_workspace_size(shape), 1), dtype=torch.uint8, device="cuda")
+    o = torch.empty_like(x["v"])
+    S_T = torch.empty_like(x["S0"])
+
+    def fn():
+        kda.kda_chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["S0"], cu, o=o, S_T=S_T, workspace=ws)
+
+    progress(f"{wname}: timing {steps} calls")
+    with ClockSampler(local) as clk:
+        t = timed(fn, steps, warmup, world, stream)
+    err = kda.kda_check_device_error()
+    if err != 0:
+        raise RuntimeError(f"device error {err} during {wname}")
+    tokens = w.B * w.T
+    ms = t / steps * 1e3
+    nbytes = prefill_bytes(tokens, 1, w.H, w.dk) - 2 * tokens * w.H * w.dk * w.dk * 4 + 2 * N * w.H * w.dk * w.dk * 4
+    flops = prefill_flops(tokens, 1, w.H, w.dk)
+    gbs = nbytes / (ms / 1e3) / 1e9
+    peak = float(peaks["hbm_gbs"])
+    c = counters.get(wname, {})
+    traffic = c.get("dram_bytes")
+    progress(f"{wname}: {ms:.3f} ms/call, {gbs:.0f} GB/s")
+    out = {
+        "value": tokens * world * steps / t, "unit": "tokens/s", "ms_per_step": ms, "steps": steps,
+        "config": {"workload": f"{wname} {w.B}x{w.T} tokens H{w.H} dk=dv={w.dk} C64, bf16 q/k/v/gates, fp32 state",
+                   "sequences": N, "tokens": tokens, "H": w.H,
+                   "l2": f"inputs larger than L2 (no flush): {tokens * w.H * w.dk * 8 / 1e6:.0f} MB read per call"},
+        "roofline": {"kernel": "kda_prefill_kernel (one cooperative launch per call)", "bound": "hbm",
+                     "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+                     "traffic": traffic, "algorithmic_bytes_per_launch": nbytes, "peak_source": peak_src,
+                     "tensor": {"achieved_tflops": flops / (ms / 1e3) / 1e12, "peak_tflops": float(peaks["bf16_tflops"]),
+                                "frac": flops / (ms / 1e3) / 1e12 / float(peaks["bf16_tflops"]),
+                                "pipe_active_pct_ncu": c.get("tensor_pipe_pct")}},
+        "clocks": clk.summary(),
+    }
+    del x, ws, o, S_T
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args):
     world, rank, local = dist_setup()
     import gated_delta_rule_110_b200 as kda
@@ -271,8 +361,13 @@ def run_ours(args):
     kda.load_library()
     peaks, peak_src = load_peaks()
     stream = torch.cuda.current_stream()
+    counters = profiled_counters()
+    launches = 0
 
-    # ---------------- prefill
+    # ---------------- prefill (the headline line)
+    pre = prefill_leg(kda, gen, "prefill", args.steps, args.warmup, world, rank, local, stream, peaks, peak_src,
+                      counters)
+    launches += args.steps
     w = gen.workload("prefill")
     x = gen.workload_inputs(w, device="cuda", seed_offset=rank)
     B, T, H, d = w.B, w.T, w.H, w.dk
@@ -280,24 +375,7 @@ def run_ours(args):
     ws = torch.empty(kda.kda_chunk_fwd_workspace_size(shape), dtype=torch.uint8, device="cuda")
     o = torch.empty_like(x["v"])
     S_T = torch.empty_like(x["S0"])
-
-    def prefill():
-        kda.kda_chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["S0"], o=o, S_T=S_T, workspace=ws)
-
-    progress("prefill: timing")
-    with ClockSampler(local) as clk:
-        t_pre = timed(prefill, args.steps, args.warmup, world, stream)
-    progress(f"prefill: {t_pre / args.steps * 1e3:.3f} ms/step")
-    err = kda.kda_check_device_error()
-    if err != 0:
-        raise RuntimeError(f"device error {err} during prefill")
     tokens_per_step = B * T
-    pre_ms = t_pre / args.steps * 1e3
-    pre_bytes = prefill_bytes(B, T, H, d)
-    pre_flops = prefill_flops(B, T, H, d)
-    value = tokens_per_step * world * args.steps / t_pre
-    achieved_gbs = pre_bytes / (pre_ms / 1e3) / 1e9
-    peak_hbm = float(peaks["hbm_gbs"])
 
     # ---------------- e2e: pinned host inputs -> device -> call -> host
     hx = {kk: x[kk].cpu().pin_memory() for kk in ("q", "k", "v", "log_alpha", "beta", "S0")}
@@ -318,8 +396,19 @@ def run_ours(args):
     progress("e2e: timing")
     e2e_steps = max(3, min(args.steps, 10))
     t_e2e = timed(e2e_step, e2e_steps, max(1, min(args.warmup, 3)), world, stream)
+    launches += e2e_steps
     e2e_value = tokens_per_step * world * e2e_steps / t_e2e
-    del dx, hx
+    del dx, hx, x, ws, o, S_T
+    torch.cuda.empty_cache()
+
+    # ---------------- varlen and long-context prefill
+    var = prefill_leg(kda, gen, "varlen", args.steps, args.warmup, world, rank, local, stream, peaks, peak_src,
+                      counters)
+    launches += args.steps
+    long_steps = max(3, min(args.steps, 5))
+    lng = prefill_leg(kda, gen, "long", long_steps, args.warmup, world, rank, local, stream, peaks, peak_src,
+                      counters)
+    launches += long_steps
 
     # ---------------- decode
     progress("decode: setup")
@@ -339,50 +428,45 @@ def run_ours(args):
     dec_steps = args.decode_steps
     with ClockSampler(local) as clk_d:
         t_dec = timed(decode, dec_steps, max(args.warmup, 3), world, stream)
+    launches += dec_steps
     err = kda.kda_check_device_error()
     if err != 0:
         raise RuntimeError(f"device error {err} during decode")
     dec_ms = t_dec / dec_steps * 1e3
     dec_bytes = decode_bytes(Nd, Hd, d)
     dec_gbs = dec_bytes / (dec_ms / 1e3) / 1e9
+    peak_hbm = float(peaks["hbm_gbs"])
+    progress(f"decode: {dec_ms:.3f} ms/step")
 
-    progress(f"decode: {t_dec / dec_steps * 1e3:.3f} ms/step")
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         progress("cpu baseline")
         cpu = oracle_baseline(w)
+        cpu["cpu_model"] = cpu_model()
 
-    clocks = clk.summary()
-    clocks_dec = clk_d.summary()
     if rank == 0:
         line = {
-            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": pre_ms, "higher_is_better": True, "scaling": "weak",
+            "metric": METRIC, "value": pre["value"], "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": pre["ms_per_step"], "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": "prefill B4 H16 T4096 dk=dv=128 C64, bf16 q/k/v/gates, fp32 state",
-                       "B": B, "T": T, "H": H, "dk": d, "dv": d, "chunk": 64,
-                       "l2": "inputs larger than L2 (no flush): 336 MB per step",
-                       "parallelism": f"weak x{world}: each rank its own workload, no collective"},
-            "roofline": {"kernel": "kda_chunk_fused_kernel (one launch per call)", "bound": "hbm",
-                         "achieved": achieved_gbs, "peak": peak_hbm, "unit": "GB/s",
-                         "frac": achieved_gbs / peak_hbm, "traffic": None,
-                         "algorithmic_bytes_per_launch": pre_bytes, "peak_source": peak_src,
-                         "tensor": {"achieved_tflops": pre_flops / (pre_ms / 1e3) / 1e12,
-                                    "peak_tflops": float(peaks["bf16_tflops"]),
-                                    "frac": pre_flops / (pre_ms / 1e3) / 1e12 / float(peaks["bf16_tflops"])}},
+            "config": dict(pre["config"], B=B, T=T, chunk=64,
+                           parallelism=f"weak x{world}: each rank its own workload, no collective"),
+            "roofline": pre["roofline"],
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": e2e_steps},
-            "gpu_launches": (args.steps + e2e_steps) + dec_steps,
-            "clocks": clocks,
+            "gpu_launches": launches,
+            "clocks": pre["clocks"],
+            "varlen": var,
+            "long": lng,
             "decode": {"value": world * dec_steps / t_dec, "unit": "steps/s", "ms_per_step": dec_ms,
                        "steps": dec_steps,
                        "config": {"workload": "decode 256 seqs x H32 dk=dv=128, fp32 state 537 MB in place, "
                                               "bf16 q/k/v/gates", "N": Nd, "H": Hd, "dk": d, "dv": d},
                        "roofline": {"kernel": "kda_decode_kernel", "bound": "hbm", "achieved": dec_gbs,
                                     "peak": peak_hbm, "unit": "GB/s", "frac": dec_gbs / peak_hbm,
-                                    "traffic": None, "algorithmic_bytes_per_launch": dec_bytes,
-                                    "peak_source": peak_src},
-                       "clocks": clocks_dec},
+                                    "traffic": counters.get("decode", {}).get("dram_bytes"),
+                                    "algorithmic_bytes_per_launch": dec_bytes, "peak_source": peak_src},
+                       "clocks": clk_d.summary()},
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
