@@ -12,6 +12,11 @@ Entry points (same names as the C ABI):
   chunkwise-parallel prefill -> ``(o, S_T)``
 * ``kda_decode_step(q, k, v, log_alpha, beta, S)`` one recurrent token per
   (sequence, head), ``S`` updated in place -> ``o``
+* ``kda_chunk_fwd_slots(q, k, v, log_alpha, beta, state_pool, state_slots,
+  has_initial_state=None, cu_seqlens=None)`` prefill reading and writing the
+  states in place in a slot-indexed pool -> ``o``
+* ``kda_decode_step_slots(q, k, v, log_alpha, beta, state_pool, state_slots)``
+  decode step on a slot-indexed pool -> ``o``
 * ``kda_chunk_fwd_workspace_size(...)``, ``kda_check_device_error()``,
   ``kda_status_string(code)``, ``kda_abi_version()``
 """
@@ -26,7 +31,7 @@ LIB_PATH = _PKG / "libkda.so"
 KDA_OK = 0
 KDA_F32, KDA_BF16 = 0, 1
 KDA_FLAG_VALIDATE_CU_SEQLENS = 0x1
-KDA_FLAG_PATH_TWO_PASS = 0x2
+KDA_FLAG_PATH_RECURRENT = 0x4
 
 _STATUS_NAMES = {
     0: "KDA_OK", -1: "KDA_ERR_NULL", -2: "KDA_ERR_SHAPE", -3: "KDA_ERR_DTYPE", -4: "KDA_ERR_ALIGN",
@@ -35,8 +40,9 @@ _STATUS_NAMES = {
 }
 
 EXPORTED_SYMBOLS = (
-    "kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_chunk_fwd_noalloc", "kda_decode_step",
-    "kda_check_device_error", "kda_status_string", "kda_abi_version",
+    "kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_chunk_fwd_noalloc", "kda_chunk_fwd_slots",
+    "kda_decode_step", "kda_decode_step_slots", "kda_check_device_error", "kda_status_string",
+    "kda_abi_version",
 )
 
 
@@ -80,8 +86,13 @@ def load_library(build_if_missing: bool = True):
     lib.kda_chunk_fwd.restype = ctypes.c_int
     lib.kda_chunk_fwd_noalloc.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.kda_chunk_fwd_noalloc.restype = ctypes.c_int
+    lib.kda_chunk_fwd_slots.argtypes = [sp, vp, vp, vp, vp, vp, vp, ctypes.c_int32, vp, vp, vp, vp, vp,
+                                        ctypes.c_size_t, vp]
+    lib.kda_chunk_fwd_slots.restype = ctypes.c_int
     lib.kda_decode_step.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.kda_decode_step.restype = ctypes.c_int
+    lib.kda_decode_step_slots.argtypes = [sp, vp, vp, vp, vp, vp, vp, ctypes.c_int32, vp, vp, vp]
+    lib.kda_decode_step_slots.restype = ctypes.c_int
     lib.kda_check_device_error.argtypes = [vp]
     lib.kda_check_device_error.restype = ctypes.c_int
     lib.kda_status_string.argtypes = [ctypes.c_int]
@@ -144,27 +155,28 @@ def tuning_flags(state_ctas: int = 0, grid_ctas: int = 0) -> int:
     return (state_ctas << 8) | (grid_ctas << 16)
 
 
-def _shape_of(q, v, log_alpha, cu_seqlens, chunk, validate, two_pass=False, state_ctas=0, grid_ctas=0):
+def _shape_of(q, v, log_alpha, cu_seqlens, chunk, validate, recurrent=False, state_ctas=0, grid_ctas=0):
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     n_seqs = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
-    flags = (KDA_FLAG_VALIDATE_CU_SEQLENS if validate else 0) | (KDA_FLAG_PATH_TWO_PASS if two_pass else 0)
+    flags = (KDA_FLAG_VALIDATE_CU_SEQLENS if validate else 0) | (KDA_FLAG_PATH_RECURRENT if recurrent else 0)
     flags |= tuning_flags(state_ctas, grid_ctas)
     return make_shape(B, T, H, dk, dv, chunk, n_seqs, _dtype_code(q), _dtype_code(log_alpha), flags)
 
 
 def kda_chunk_fwd(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, *, chunk: int = 64, o=None, S_T=None,
                   workspace=None, stream=None, validate: bool = False, output_final_state: bool = True,
-                  two_pass: bool = False, state_ctas: int = 0, grid_ctas: int = 0):
+                  recurrent: bool = False, state_ctas: int = 0, grid_ctas: int = 0):
     """Chunkwise KDA prefill.  Shapes as in include/kda.h; returns (o, S_T).
 
     The tensor-core path needs a workspace (allocated here from PyTorch's
-    caching allocator if not given).  ``two_pass=True`` selects the prep +
-    recurrence kernels instead of the default pipelined kernel;
-    ``state_ctas`` / ``grid_ctas`` override its CTA split (0 = automatic)."""
+    caching allocator if not given).  ``recurrent=True`` runs the fp32
+    token-by-token CUDA-core recurrence instead (a reference path);
+    ``state_ctas`` / ``grid_ctas`` override the tensor-core path's CTA split
+    (0 = automatic)."""
     import torch
     _need_cuda(q, k, v, log_alpha, beta, S0, cu_seqlens, o, S_T, workspace)
-    shape = _shape_of(q, v, log_alpha, cu_seqlens, chunk, validate, two_pass, state_ctas, grid_ctas)
+    shape = _shape_of(q, v, log_alpha, cu_seqlens, chunk, validate, recurrent, state_ctas, grid_ctas)
     N = shape.B if cu_seqlens is None else shape.n_seqs
     if o is None:
         o = torch.empty(v.shape, dtype=v.dtype, device=v.device)
@@ -183,7 +195,7 @@ def kda_chunk_fwd(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, *, chunk: 
 
 
 def kda_chunk_fwd_noalloc(q, k, v, log_alpha, beta, S0, cu_seqlens, o, S_T, *, chunk: int = 64, stream=None,
-                          two_pass: bool = False):
+                          state_ctas: int = 0, grid_ctas: int = 0):
     """kda_chunk_fwd on the library's built-in scratch array (no workspace).
 
     For callers that cannot allocate device memory where they run the prefill
@@ -191,13 +203,73 @@ def kda_chunk_fwd_noalloc(q, k, v, log_alpha, beta, S0, cu_seqlens, o, S_T, *, c
     are caller-owned outputs; nothing is allocated here.
     """
     _need_cuda(q, k, v, log_alpha, beta, S0, cu_seqlens, o, S_T)
-    shape = _shape_of(q, v, log_alpha, cu_seqlens, chunk, False, two_pass)
+    shape = _shape_of(q, v, log_alpha, cu_seqlens, chunk, False, False, state_ctas, grid_ctas)
     rc = load_library().kda_chunk_fwd_noalloc(
         ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0),
         _ptr(cu_seqlens), _ptr(o), _ptr(S_T), _stream(stream))
     if rc != KDA_OK:
         raise KdaError(rc, "kda_chunk_fwd_noalloc")
     return o, S_T
+
+
+def _check_slots(state_pool, state_slots, n, has_initial_state=None):
+    import torch
+    if state_pool.dtype != torch.float32 or state_pool.dim() != 4:
+        raise ValueError("state_pool must be a [num_slots, H, dk, dv] float32 tensor")
+    if state_slots.dtype != torch.int32 or state_slots.numel() != n:
+        raise ValueError(f"state_slots must be an int32 tensor with one entry per sequence ({n})")
+    if has_initial_state is not None and (has_initial_state.dtype not in (torch.uint8, torch.bool)
+                                          or has_initial_state.numel() != n):
+        raise ValueError(f"has_initial_state must be a uint8/bool tensor with one entry per sequence ({n})")
+
+
+def kda_chunk_fwd_slots(q, k, v, log_alpha, beta, state_pool, state_slots, has_initial_state=None,
+                        cu_seqlens=None, *, chunk: int = 64, o=None, workspace=None, stream=None,
+                        validate: bool = False, recurrent: bool = False, state_ctas: int = 0,
+                        grid_ctas: int = 0):
+    """Prefill on a slot-indexed state pool (include/kda.h, serving-state
+    variants).  Sequence n starts from ``state_pool[state_slots[n]]`` (or from
+    zeros where ``has_initial_state[n]`` is 0) and its final state is written
+    back there; a negative slot is padding (zero start, state dropped).
+    Returns o."""
+    import torch
+    _need_cuda(q, k, v, log_alpha, beta, state_pool, state_slots, has_initial_state, cu_seqlens, o, workspace)
+    shape = _shape_of(q, v, log_alpha, cu_seqlens, chunk, validate, recurrent, state_ctas, grid_ctas)
+    N = shape.B if cu_seqlens is None else shape.n_seqs
+    _check_slots(state_pool, state_slots, N, has_initial_state)
+    if o is None:
+        o = torch.empty(v.shape, dtype=v.dtype, device=v.device)
+    need = kda_chunk_fwd_workspace_size(shape)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = load_library().kda_chunk_fwd_slots(
+        ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(state_pool),
+        int(state_pool.shape[0]), _ptr(state_slots), _ptr(has_initial_state), _ptr(cu_seqlens), _ptr(o),
+        _ptr(workspace), ws_bytes, _stream(stream))
+    if rc != KDA_OK:
+        raise KdaError(rc, "kda_chunk_fwd_slots")
+    return o
+
+
+def kda_decode_step_slots(q, k, v, log_alpha, beta, state_pool, state_slots, *, o=None, stream=None):
+    """One recurrent token per row on a slot-indexed state pool: row n updates
+    ``state_pool[state_slots[n]]`` in place (negative slot: padding, zero
+    state, nothing written).  Returns o [N,H,dv]."""
+    import torch
+    _need_cuda(q, k, v, log_alpha, beta, state_pool, state_slots, o)
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    _check_slots(state_pool, state_slots, N)
+    shape = make_shape(N, 1, H, dk, dv, 64, 0, _dtype_code(q), _dtype_code(log_alpha), 0)
+    if o is None:
+        o = torch.empty(v.shape, dtype=v.dtype, device=v.device)
+    rc = load_library().kda_decode_step_slots(
+        ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(state_pool),
+        int(state_pool.shape[0]), _ptr(state_slots), _ptr(o), _stream(stream))
+    if rc != KDA_OK:
+        raise KdaError(rc, "kda_decode_step_slots")
+    return o
 
 
 def kda_decode_step(q, k, v, log_alpha, beta, S, *, o=None, stream=None):

@@ -9,15 +9,11 @@
 #include <vector>
 
 #include "kda.h"
-#include "kda_chunk_tc.cuh"
 #include "kda_prefill.cuh"
 #include "kda_recurrent.cuh"
 #include "kda_tma.h"
 
 namespace {
-
-using kda::tc::C;
-using kda::tc::SLOT_BYTES;
 
 inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 inline bool aligned16(const void* p) { return aligned(p, 16); }
@@ -32,16 +28,13 @@ inline bool token_ptrs_aligned(const kda_shape& s, const void* q, const void* k,
 inline bool dtype_ok(int32_t d) { return d == KDA_F32 || d == KDA_BF16; }
 inline bool dim_ok(int32_t d) { return d == 64 || d == 128; }
 
-// Tensor-core chunk path: bf16 io, dk = dv = 128, C = 64.  It runs the
-// pipelined kernel (state CTAs + transform CTAs through an L2-resident ring)
-// unless KDA_FLAG_PATH_TWO_PASS asks for the two-kernel form (prep + recurrence
-// through a workspace holding every chunk's operands).
+// Tensor-core chunk path: bf16 io and dk = dv = 128 (chunk C = 64), unless
+// KDA_FLAG_PATH_RECURRENT asks for the token-by-token CUDA-core recurrence.
 inline bool use_tc(const kda_shape& s) {
-  return s.io_dtype == KDA_BF16 && s.dk == 128 && s.dv == 128 && s.chunk == 64;
+  return s.io_dtype == KDA_BF16 && s.dk == 128 && s.dv == 128 && (s.flags & KDA_FLAG_PATH_RECURRENT) == 0u;
 }
-inline bool use_two_pass(const kda_shape& s) { return use_tc(s) && (s.flags & KDA_FLAG_PATH_TWO_PASS) != 0u; }
 constexpr uint32_t kKnownFlags =
-    KDA_FLAG_VALIDATE_CU_SEQLENS | KDA_FLAG_PATH_TWO_PASS | KDA_FLAG_STATE_CTAS(0xFF) | KDA_FLAG_GRID_CTAS(0xFF);
+    KDA_FLAG_VALIDATE_CU_SEQLENS | KDA_FLAG_PATH_RECURRENT | KDA_FLAG_STATE_CTAS(0xFF) | KDA_FLAG_GRID_CTAS(0xFF);
 
 // Number of sequences N and the packed token total.
 inline void seq_counts(const kda_shape& s, const int32_t* cu, int64_t* N, int64_t* Ttot) {
@@ -53,10 +46,6 @@ inline void seq_counts(const kda_shape& s, const int32_t* cu, int64_t* N, int64_
     *Ttot = static_cast<int64_t>(s.B) * s.T;
   }
 }
-
-// Upper bound on the number of chunks over all sequences: each sequence of
-// length l has ceil(l / C) <= l / C + 1 chunks.
-inline int64_t max_chunks(int64_t N, int64_t Ttot) { return Ttot / C + N; }
 
 kda_status check_common(const kda_shape* sp) {
   if (!sp) return KDA_ERR_NULL;
@@ -75,45 +64,47 @@ kda_status launch_status() {
 
 template <int DK, int DV, typename TIO, typename TG>
 kda_status launch_recurrent_fwd(const kda_shape& s, int64_t N, const void* q, const void* k, const void* v,
-                                const void* la, const void* beta, const float* S0, const int32_t* cu, void* o,
-                                float* S_T, cudaStream_t st) {
+                                const void* la, const void* beta, const kda::StateIO& io, const int32_t* cu,
+                                void* o, cudaStream_t st) {
   dim3 grid(s.H, static_cast<unsigned>(N));
   kda::kda_recurrent_fwd_kernel<DK, DV, TIO, TG><<<grid, kda::kRecThreads, 0, st>>>(
       s.H, s.T, cu, static_cast<const TIO*>(q), static_cast<const TIO*>(k), static_cast<const TIO*>(v),
-      static_cast<const TG*>(la), static_cast<const TG*>(beta), S0, static_cast<TIO*>(o), S_T);
+      static_cast<const TG*>(la), static_cast<const TG*>(beta), io, static_cast<TIO*>(o));
   return launch_status();
 }
 
 template <typename TIO, typename TG>
 kda_status dispatch_recurrent_fwd(const kda_shape& s, int64_t N, const void* q, const void* k, const void* v,
-                                  const void* la, const void* beta, const float* S0, const int32_t* cu, void* o,
-                                  float* S_T, cudaStream_t st) {
+                                  const void* la, const void* beta, const kda::StateIO& io, const int32_t* cu,
+                                  void* o, cudaStream_t st) {
   if (s.dk == 128 && s.dv == 128)
-    return launch_recurrent_fwd<128, 128, TIO, TG>(s, N, q, k, v, la, beta, S0, cu, o, S_T, st);
+    return launch_recurrent_fwd<128, 128, TIO, TG>(s, N, q, k, v, la, beta, io, cu, o, st);
   if (s.dk == 64 && s.dv == 64)
-    return launch_recurrent_fwd<64, 64, TIO, TG>(s, N, q, k, v, la, beta, S0, cu, o, S_T, st);
+    return launch_recurrent_fwd<64, 64, TIO, TG>(s, N, q, k, v, la, beta, io, cu, o, st);
   if (s.dk == 128 && s.dv == 64)
-    return launch_recurrent_fwd<128, 64, TIO, TG>(s, N, q, k, v, la, beta, S0, cu, o, S_T, st);
-  return launch_recurrent_fwd<64, 128, TIO, TG>(s, N, q, k, v, la, beta, S0, cu, o, S_T, st);
+    return launch_recurrent_fwd<128, 64, TIO, TG>(s, N, q, k, v, la, beta, io, cu, o, st);
+  return launch_recurrent_fwd<64, 128, TIO, TG>(s, N, q, k, v, la, beta, io, cu, o, st);
 }
 
 template <int DK, int DV, typename TIO, typename TG>
 kda_status launch_decode(const kda_shape& s, const void* q, const void* k, const void* v, const void* la,
-                         const void* beta, float* S, void* o, cudaStream_t st) {
+                         const void* beta, float* S, const int32_t* slots, int num_slots, void* o,
+                         cudaStream_t st) {
   const unsigned blocks = static_cast<unsigned>(s.B) * static_cast<unsigned>(s.H);
   kda::kda_decode_kernel<DK, DV, TIO, TG><<<blocks, kda::kRecThreads, 0, st>>>(
       s.H, static_cast<const TIO*>(q), static_cast<const TIO*>(k), static_cast<const TIO*>(v),
-      static_cast<const TG*>(la), static_cast<const TG*>(beta), S, static_cast<TIO*>(o));
+      static_cast<const TG*>(la), static_cast<const TG*>(beta), S, static_cast<TIO*>(o), slots, num_slots);
   return launch_status();
 }
 
 template <typename TIO, typename TG>
 kda_status dispatch_decode(const kda_shape& s, const void* q, const void* k, const void* v, const void* la,
-                           const void* beta, float* S, void* o, cudaStream_t st) {
-  if (s.dk == 128 && s.dv == 128) return launch_decode<128, 128, TIO, TG>(s, q, k, v, la, beta, S, o, st);
-  if (s.dk == 64 && s.dv == 64) return launch_decode<64, 64, TIO, TG>(s, q, k, v, la, beta, S, o, st);
-  if (s.dk == 128 && s.dv == 64) return launch_decode<128, 64, TIO, TG>(s, q, k, v, la, beta, S, o, st);
-  return launch_decode<64, 128, TIO, TG>(s, q, k, v, la, beta, S, o, st);
+                           const void* beta, float* S, const int32_t* slots, int num_slots, void* o,
+                           cudaStream_t st) {
+  if (s.dk == 128 && s.dv == 128) return launch_decode<128, 128, TIO, TG>(s, q, k, v, la, beta, S, slots, num_slots, o, st);
+  if (s.dk == 64 && s.dv == 64) return launch_decode<64, 64, TIO, TG>(s, q, k, v, la, beta, S, slots, num_slots, o, st);
+  if (s.dk == 128 && s.dv == 64) return launch_decode<128, 64, TIO, TG>(s, q, k, v, la, beta, S, slots, num_slots, o, st);
+  return launch_decode<64, 128, TIO, TG>(s, q, k, v, la, beta, S, slots, num_slots, o, st);
 }
 
 // Opt-in to large dynamic shared memory.  Set on every launch: the call is
@@ -123,30 +114,6 @@ template <typename F>
 bool ensure_smem(F* kernel, uint32_t bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes)) ==
          cudaSuccess;
-}
-
-template <typename TG>
-kda_status launch_tc(const kda_shape& s, int64_t N, int64_t Ttot, const void* q, const void* k, const void* v,
-                     const void* la, const void* beta, const float* S0, const int32_t* cu, void* o, float* S_T,
-                     void* ws, cudaStream_t st) {
-  auto* prep = kda::tc::kda_chunk_prep_kernel<TG>;
-  auto* rec = kda::tc::kda_chunk_rec_kernel<__nv_bfloat16>;
-  if (!ensure_smem(prep, kda::tc::P_SMEM) || !ensure_smem(rec, kda::tc::R_SMEM)) return KDA_ERR_CUDA;
-  const int64_t mc = max_chunks(N, Ttot);
-  if (mc > 0) {
-    dim3 g1(static_cast<unsigned>(mc), static_cast<unsigned>(s.H));
-    prep<<<g1, 256, kda::tc::P_SMEM, st>>>(static_cast<int>(N), s.T, s.H, cu,
-                                           static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-                                           static_cast<const __nv_bfloat16*>(v), static_cast<const TG*>(la),
-                                           static_cast<const TG*>(beta), static_cast<uint8_t*>(ws));
-    const kda_status e = launch_status();
-    if (e != KDA_OK) return e;
-  }
-  dim3 g2(static_cast<unsigned>(s.H), static_cast<unsigned>(N));
-  rec<<<g2, kda::tc::REC_THREADS, kda::tc::R_SMEM, st>>>(static_cast<int>(N), s.T, s.H, cu,
-                                                         static_cast<const uint8_t*>(ws), S0,
-                                                         static_cast<__nv_bfloat16*>(o), S_T);
-  return launch_status();
 }
 
 // ---------------------------------------------------------------------------
@@ -164,7 +131,15 @@ struct PrefillPlan {
   int grid = 0;          // all CTAs (one per SM)
   size_t flag_bytes = 0; // zeroed before each launch
   size_t ring_off = 0;
-  size_t bytes = 0;      // workspace
+  size_t ring_unit = 0;  // bytes per ring slot of every state CTA
+  size_t bytes = 0;      // preferred workspace: the deepest ring
+  size_t min_bytes = 0;  // smallest usable workspace: a 2-slot ring
+  // ring depth a workspace of ws_bytes allows (0 if too small)
+  int nring(size_t ws_bytes) const {
+    if (ws_bytes < min_bytes) return 0;
+    const size_t d = (ws_bytes - ring_off) / ring_unit;
+    return static_cast<int>(d < static_cast<size_t>(kda::pipe::MAX_RING) ? d : kda::pipe::MAX_RING);
+  }
 };
 
 // Splits the SMs between state CTAs (one serial chain of chunks each) and
@@ -202,18 +177,21 @@ PrefillPlan plan_prefill(const kda_shape& s, int64_t N, int nsm) {
   pl.grid = grid;
   pl.flag_bytes = kda::pipe::flag_words(R) * sizeof(uint32_t);
   pl.ring_off = (pl.flag_bytes + 1023) & ~static_cast<size_t>(1023);
-  pl.bytes = pl.ring_off + static_cast<size_t>(R) * kda::pipe::NRING * kda::pipe::SLOT;
+  pl.ring_unit = static_cast<size_t>(R) * kda::pipe::SLOT;
+  pl.bytes = pl.ring_off + pl.ring_unit * kda::pipe::MAX_RING;
+  pl.min_bytes = pl.ring_off + pl.ring_unit * 2;
   return pl;
 }
 
 template <typename TG>
 kda_status launch_prefill(const kda_shape& s, int64_t N, int64_t Ttot, const void* q, const void* k, const void* v,
-                          const void* la, const void* beta, const float* S0, const int32_t* cu, void* o, float* S_T,
+                          const void* la, const void* beta, const kda::StateIO& io, const int32_t* cu, void* o,
                           void* ws, size_t ws_bytes, cudaStream_t st) {
   namespace P = kda::pipe;
   const PrefillPlan pl = plan_prefill(s, N, device_sm_count());
   if (pl.R <= 0) return KDA_ERR_CUDA;
-  if (!ws || ws_bytes < pl.bytes) return KDA_ERR_WORKSPACE;
+  const int nring = pl.nring(ws_bytes);
+  if (!ws || nring < 2) return KDA_ERR_WORKSPACE;
   // the work-item counter is 32-bit: R * (chunks of the longest stream) must fit
   if (static_cast<double>(pl.R) * (static_cast<double>(Ttot) / P::C + static_cast<double>(N)) > 2.0e9)
     return KDA_ERR_SHAPE;
@@ -234,11 +212,11 @@ kda_status launch_prefill(const kda_shape& s, int64_t N, int64_t Ttot, const voi
   prm.H = s.H;
   prm.N = static_cast<int>(N);
   prm.R = pl.R;
+  prm.nring = nring;
   prm.cu = cu;
   prm.beta = beta;
-  prm.S0 = S0;
+  prm.st = io;
   prm.o = static_cast<__nv_bfloat16*>(o);
-  prm.S_T = S_T;
   prm.flags = static_cast<uint32_t*>(ws);
   prm.ring = static_cast<uint8_t*>(ws) + pl.ring_off;
   auto* kern = P::kda_prefill_kernel<TG>;
@@ -283,24 +261,38 @@ size_t kda_chunk_fwd_workspace_size(const kda_shape* sp) {
   if (!use_tc(s)) return 0;
   const bool packed = s.n_seqs > 0 && s.B == 1;
   const int64_t N = packed ? s.n_seqs : s.B;
-  const int64_t Ttot = packed ? s.T : static_cast<int64_t>(s.B) * s.T;
-  if (use_two_pass(s)) return static_cast<size_t>(max_chunks(N, Ttot)) * static_cast<size_t>(s.H) * SLOT_BYTES;
   return plan_prefill(s, N, device_sm_count()).bytes;
 }
 
-kda_status kda_chunk_fwd(const kda_shape* sp, const void* q, const void* k, const void* v, const void* log_alpha,
-                         const void* beta, const float* S0, const int32_t* cu_seqlens, void* o, float* S_T,
-                         void* workspace, size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+// Smallest workspace kda_chunk_fwd accepts: the pipelined path runs with any
+// ring depth from 2 to 16 slots per state CTA.
+size_t kda_chunk_fwd_min_workspace(const kda_shape* sp) {
+  if (check_common(sp) != KDA_OK) return 0;
+  const kda_shape& s = *sp;
+  if (!use_tc(s)) return 0;
+  const bool packed = s.n_seqs > 0 && s.B == 1;
+  const int64_t N = packed ? s.n_seqs : s.B;
+  return plan_prefill(s, N, device_sm_count()).min_bytes;
+}
+
+// Shared body of kda_chunk_fwd and kda_chunk_fwd_slots; `io` says where the
+// states live (dense rows or pool slots).
+kda_status chunk_fwd(const kda_shape* sp, const void* q, const void* k, const void* v, const void* log_alpha,
+                     const void* beta, const kda::StateIO& io, const int32_t* cu_seqlens, void* o, void* workspace,
+                     size_t workspace_bytes, void* stream) {
   kda_status e = check_common(sp);
   if (e != KDA_OK) return e;
   const kda_shape& s = *sp;
-  if (s.chunk != 16 && s.chunk != 32 && s.chunk != 64) return KDA_ERR_UNSUPPORTED;
+  if (s.chunk != 64) return KDA_ERR_UNSUPPORTED;
   if (cu_seqlens && (s.B != 1 || s.n_seqs <= 0)) return KDA_ERR_SHAPE;
   int64_t N, Ttot;
   seq_counts(s, cu_seqlens, &N, &Ttot);
   const bool any_tokens = Ttot > 0;
   if (any_tokens && (!q || !k || !v || !log_alpha || !beta || !o)) return KDA_ERR_NULL;
-  if (!token_ptrs_aligned(s, q, k, v, log_alpha, beta, o) || !aligned16(S0) || !aligned16(S_T) ||
+  if (!token_ptrs_aligned(s, q, k, v, log_alpha, beta, o) || !aligned16(io.S0) || !aligned16(io.S_T) ||
       !aligned(cu_seqlens, 4))
     return KDA_ERR_ALIGN;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -310,52 +302,89 @@ kda_status kda_chunk_fwd(const kda_shape* sp, const void* q, const void* k, cons
   }
   if (N == 0) return KDA_OK;
 
-  if (use_tc(s) && !use_two_pass(s) && Ttot > 0) {
+  if (use_tc(s) && Ttot > 0) {
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(log_alpha) || !aligned16(o))
       return KDA_ERR_ALIGN;
     if (s.gate_dtype == KDA_BF16)
-      return launch_prefill<__nv_bfloat16>(s, N, Ttot, q, k, v, log_alpha, beta, S0, cu_seqlens, o, S_T, workspace,
+      return launch_prefill<__nv_bfloat16>(s, N, Ttot, q, k, v, log_alpha, beta, io, cu_seqlens, o, workspace,
                                            workspace_bytes, st);
-    return launch_prefill<float>(s, N, Ttot, q, k, v, log_alpha, beta, S0, cu_seqlens, o, S_T, workspace,
+    return launch_prefill<float>(s, N, Ttot, q, k, v, log_alpha, beta, io, cu_seqlens, o, workspace,
                                  workspace_bytes, st);
-  }
-  if (use_two_pass(s)) {
-    const size_t need = kda_chunk_fwd_workspace_size(sp);
-    if (need > 0 && (!workspace || workspace_bytes < need)) return KDA_ERR_WORKSPACE;
-    if (!aligned16(workspace)) return KDA_ERR_ALIGN;
-    if (s.gate_dtype == KDA_BF16)
-      return launch_tc<__nv_bfloat16>(s, N, Ttot, q, k, v, log_alpha, beta, S0, cu_seqlens, o, S_T, workspace, st);
-    return launch_tc<float>(s, N, Ttot, q, k, v, log_alpha, beta, S0, cu_seqlens, o, S_T, workspace, st);
   }
   if (s.io_dtype == KDA_F32) {
     if (s.gate_dtype == KDA_F32)
-      return dispatch_recurrent_fwd<float, float>(s, N, q, k, v, log_alpha, beta, S0, cu_seqlens, o, S_T, st);
-    return dispatch_recurrent_fwd<float, __nv_bfloat16>(s, N, q, k, v, log_alpha, beta, S0, cu_seqlens, o, S_T,
-                                                         st);
+      return dispatch_recurrent_fwd<float, float>(s, N, q, k, v, log_alpha, beta, io, cu_seqlens, o, st);
+    return dispatch_recurrent_fwd<float, __nv_bfloat16>(s, N, q, k, v, log_alpha, beta, io, cu_seqlens, o, st);
   }
   if (s.gate_dtype == KDA_F32)
-    return dispatch_recurrent_fwd<__nv_bfloat16, float>(s, N, q, k, v, log_alpha, beta, S0, cu_seqlens, o, S_T,
-                                                        st);
-  return dispatch_recurrent_fwd<__nv_bfloat16, __nv_bfloat16>(s, N, q, k, v, log_alpha, beta, S0, cu_seqlens, o,
-                                                              S_T, st);
+    return dispatch_recurrent_fwd<__nv_bfloat16, float>(s, N, q, k, v, log_alpha, beta, io, cu_seqlens, o, st);
+  return dispatch_recurrent_fwd<__nv_bfloat16, __nv_bfloat16>(s, N, q, k, v, log_alpha, beta, io, cu_seqlens, o,
+                                                              st);
 }
 
-kda_status kda_decode_step(const kda_shape* sp, const void* q, const void* k, const void* v, const void* log_alpha,
-                           const void* beta, float* S, void* o, void* stream) {
+// Shared body of kda_decode_step and kda_decode_step_slots.
+kda_status decode_step(const kda_shape* sp, const void* q, const void* k, const void* v, const void* log_alpha,
+                       const void* beta, float* S, const int32_t* slots, int num_slots, void* o, void* stream) {
   kda_status e = check_common(sp);
   if (e != KDA_OK) return e;
   const kda_shape& s = *sp;
   if (s.T != 1) return KDA_ERR_SHAPE;
   if (!q || !k || !v || !log_alpha || !beta || !S || !o) return KDA_ERR_NULL;
-  if (!token_ptrs_aligned(s, q, k, v, log_alpha, beta, o) || !aligned16(S)) return KDA_ERR_ALIGN;
+  if (!token_ptrs_aligned(s, q, k, v, log_alpha, beta, o) || !aligned16(S) || !aligned(slots, 4))
+    return KDA_ERR_ALIGN;
   if (static_cast<int64_t>(s.B) * s.H > 0x7fffffffLL) return KDA_ERR_SHAPE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (s.io_dtype == KDA_F32) {
-    if (s.gate_dtype == KDA_F32) return dispatch_decode<float, float>(s, q, k, v, log_alpha, beta, S, o, st);
-    return dispatch_decode<float, __nv_bfloat16>(s, q, k, v, log_alpha, beta, S, o, st);
+    if (s.gate_dtype == KDA_F32)
+      return dispatch_decode<float, float>(s, q, k, v, log_alpha, beta, S, slots, num_slots, o, st);
+    return dispatch_decode<float, __nv_bfloat16>(s, q, k, v, log_alpha, beta, S, slots, num_slots, o, st);
   }
-  if (s.gate_dtype == KDA_F32) return dispatch_decode<__nv_bfloat16, float>(s, q, k, v, log_alpha, beta, S, o, st);
-  return dispatch_decode<__nv_bfloat16, __nv_bfloat16>(s, q, k, v, log_alpha, beta, S, o, st);
+  if (s.gate_dtype == KDA_F32)
+    return dispatch_decode<__nv_bfloat16, float>(s, q, k, v, log_alpha, beta, S, slots, num_slots, o, st);
+  return dispatch_decode<__nv_bfloat16, __nv_bfloat16>(s, q, k, v, log_alpha, beta, S, slots, num_slots, o, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+kda_status kda_chunk_fwd(const kda_shape* sp, const void* q, const void* k, const void* v, const void* log_alpha,
+                         const void* beta, const float* S0, const int32_t* cu_seqlens, void* o, float* S_T,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+  kda::StateIO io;
+  io.S0 = S0;
+  io.S_T = S_T;
+  return chunk_fwd(sp, q, k, v, log_alpha, beta, io, cu_seqlens, o, workspace, workspace_bytes, stream);
+}
+
+kda_status kda_chunk_fwd_slots(const kda_shape* sp, const void* q, const void* k, const void* v,
+                               const void* log_alpha, const void* beta, float* state_pool, int32_t num_slots,
+                               const int32_t* state_slots, const uint8_t* has_initial_state,
+                               const int32_t* cu_seqlens, void* o, void* workspace, size_t workspace_bytes,
+                               void* stream) {
+  if (!state_pool || !state_slots) return KDA_ERR_NULL;
+  if (num_slots <= 0) return KDA_ERR_SHAPE;
+  if (!aligned(state_slots, 4)) return KDA_ERR_ALIGN;
+  kda::StateIO io;
+  io.S0 = state_pool;
+  io.S_T = state_pool;
+  io.slots = state_slots;
+  io.has_init = has_initial_state;
+  io.num_slots = num_slots;
+  return chunk_fwd(sp, q, k, v, log_alpha, beta, io, cu_seqlens, o, workspace, workspace_bytes, stream);
+}
+
+kda_status kda_decode_step(const kda_shape* sp, const void* q, const void* k, const void* v, const void* log_alpha,
+                           const void* beta, float* S, void* o, void* stream) {
+  return decode_step(sp, q, k, v, log_alpha, beta, S, nullptr, 0, o, stream);
+}
+
+kda_status kda_decode_step_slots(const kda_shape* sp, const void* q, const void* k, const void* v,
+                                 const void* log_alpha, const void* beta, float* state_pool, int32_t num_slots,
+                                 const int32_t* state_slots, void* o, void* stream) {
+  if (!state_slots) return KDA_ERR_NULL;
+  if (num_slots <= 0) return KDA_ERR_SHAPE;
+  return decode_step(sp, q, k, v, log_alpha, beta, state_pool, state_slots, num_slots, o, stream);
 }
 
 kda_status kda_check_device_error(void* stream) {
@@ -377,7 +406,7 @@ const char* kda_status_string(kda_status status) {
     case KDA_ERR_SHAPE: return "invalid or inconsistent sizes";
     case KDA_ERR_DTYPE: return "unknown dtype code";
     case KDA_ERR_ALIGN: return "a pointer is not aligned as required";
-    case KDA_ERR_UNSUPPORTED: return "configuration not supported (dk, dv must be 64 or 128; chunk 16, 32 or 64)";
+    case KDA_ERR_UNSUPPORTED: return "configuration not supported (dk, dv must be 64 or 128; chunk must be 64)";
     case KDA_ERR_WORKSPACE: return "workspace missing or too small";
     case KDA_ERR_CUDA: return "a CUDA runtime call or kernel launch failed";
     case KDA_ERR_TIMEOUT: return "a device-side bounded wait timed out";
@@ -422,8 +451,9 @@ extern "C" kda_status kda_chunk_fwd_noalloc(const kda_shape* sp_in, const void* 
   const kda_status e = check_common(sp_in);
   if (e != KDA_OK) return e;
   const kda_shape* sp = sp_in;
-  // an oversized request is refused before anything is launched
-  const size_t need = kda_chunk_fwd_workspace_size(sp);
+  // an oversized request is refused before anything is launched; on the
+  // pipelined path the ring is made as deep as the array allows
+  const size_t need = kda_chunk_fwd_min_workspace(sp);
   if (need > kNoAllocScratchBytes) return KDA_ERR_WORKSPACE;
   void* scratch = nullptr;
   if (need > 0) {
@@ -433,3 +463,11 @@ extern "C" kda_status kda_chunk_fwd_noalloc(const kda_shape* sp_in, const void* 
   return kda_chunk_fwd(sp, q, k, v, log_alpha, beta, S0, cu_seqlens, o, S_T, scratch,
                        need > 0 ? kNoAllocScratchBytes : 0, stream);
 }
+
+#ifdef KDA_TEST_HOOKS
+// Test-only build: arms (1) or disarms (0) the skipped completion signal of
+// g_test_skip_commit on the current device.
+extern "C" int kda_test_set_skip_commit(int on) {
+  return cudaMemcpyToSymbol(kda::pipe::g_test_skip_commit, &on, sizeof(int)) == cudaSuccess ? 0 : -1;
+}
+#endif

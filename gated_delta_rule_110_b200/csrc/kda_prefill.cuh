@@ -31,7 +31,7 @@
 //     (a tensor-core product with a lower-triangular ones matrix), the scaled
 //     tiles, A / P on tcgen05, T by blocked forward substitution on CUDA cores,
 //     W'^T on tcgen05, and write them to a ring slot in global memory.
-// The ring (NRING slots per state CTA, ~65 KB each) is small enough to stay in
+// The ring (nring <= 16 slots per state CTA, ~65 KB each) is small enough to stay in
 // L2.  A transform CTA claims work items from a global counter in stream
 // order; it writes a slot once the state CTA has copied the slot's previous
 // contents (the `consumed` counter) and publishes it with a release store of
@@ -44,14 +44,22 @@
 #pragma once
 
 #include "kda_ptx.cuh"
+#include "kda_state_io.cuh"
 
 namespace kda {
 namespace pipe {
 
+#ifdef KDA_TEST_HOOKS
+// Test-only build: when set, state CTA 0 never signals that its first U^T is
+// complete, so the state warps' bounded wait runs out (the failure-detection
+// test); every other wait then ends through the abort flag or its own limit.
+__device__ int g_test_skip_commit = 0;
+#endif
+
 constexpr int C = 64;
 constexpr int D = 128;
 constexpr int NTHREADS = 384;
-constexpr int NRING = 8;
+constexpr int MAX_RING = 16;  // ring slots per state CTA (the host picks 2..16)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kSpan2 = 230.0f;  // largest chunk decay of the factorised path, log2 units
 
@@ -67,7 +75,7 @@ constexpr uint32_t SLOT = 66560;
 // ---- global flags (32-bit words) ---------------------------------------------
 constexpr uint32_t F_COUNTER = 0;     // next work item
 constexpr uint32_t F_ABORT = 32;      // any CTA gave up
-constexpr uint32_t F_REC0 = 64;       // per state CTA: ready[NRING] at +0, consumed at +32
+constexpr uint32_t F_REC0 = 64;       // per state CTA: ready[nring] at +0, consumed at +32
 constexpr uint32_t F_REC_STRIDE = 64;
 constexpr uint32_t F_CONSUMED = 32;
 __host__ __device__ constexpr size_t flag_words(int R) { return F_REC0 + static_cast<size_t>(R) * F_REC_STRIDE; }
@@ -134,10 +142,10 @@ struct Params {
   int R;            // state CTAs
   const int32_t* cu;
   const void* beta;
-  const float* S0;
+  StateIO st;       // initial / final states (dense rows or pool slots)
   __nv_bfloat16* o;
-  float* S_T;
-  uint8_t* ring;    // R * NRING slots
+  int nring;        // ring slots per state CTA, 2..MAX_RING
+  uint8_t* ring;    // R * nring slots
   uint32_t* flags;  // flag_words(R), zero on entry
 };
 
@@ -264,7 +272,7 @@ struct Tf {
       if (prev_si < 0) return true;
       const int k = nfinished;
       if (!mbar_wait(&bars[BT_WT_STAGED], k & 1, abort_flag)) return false;
-      uint8_t* pslot = p.ring + (static_cast<size_t>(prev_si) * NRING + (prev_pos % NRING)) * SLOT;
+      uint8_t* pslot = p.ring + (static_cast<size_t>(prev_si) * p.nring + (prev_pos % p.nring)) * SLOT;
       bulk_s2g(pslot + R_WT, gb + LY::G_KB, 16384);
       bulk_commit();
       bulk_wait_read<0>();
@@ -273,7 +281,7 @@ struct Tf {
       if (!*abort_flag) {
         fence_proxy_async_global();
         __threadfence();
-        st_release_gpu(gflags + F_REC0 + prev_si * F_REC_STRIDE + (prev_pos % NRING),
+        st_release_gpu(gflags + F_REC0 + prev_si * F_REC_STRIDE + (prev_pos % p.nring),
                        static_cast<uint32_t>(prev_pos + 1));
       }
       ++nfinished;
@@ -288,6 +296,7 @@ struct Tf {
         if (it >= 1 && !mbar_wait(&bars[BT_RAW_FREE], (it - 1) & 1, abort_flag)) stop = 1;
         while (!stop && !done) {
           if (*abort_flag || *reinterpret_cast<volatile uint32_t*>(gflags + F_ABORT) != 0u) {
+            *abort_flag = 1;  // the group's other warps unwind at once
             stop = 1;
             break;
           }
@@ -362,6 +371,7 @@ struct Tf {
       if (__shfl_sync(0xffffffffu, stop, 0)) break;
     }
     if (lane == 0 && !*abort_flag) finish_prev();
+    if (lane == 0) bulk_wait_all();  // copies out of shared memory end before the CTA does
     // a load issued for an item that was never consumed must land before exit
     if (lane == 0 && it >= 1) {
       const long long t0 = clock64();
@@ -443,20 +453,23 @@ struct Tf {
       // the abort flag, and every barrier is still reached.
       const bool got = mbar_wait_warp(&bars[BT_RAW_FULL], it & 1, abort_flag);
       const bool fin = got && *reinterpret_cast<volatile int*>(&meta[MT_DONE]) != 0;
-      if (named_bar_or(1 + g, 128, !got || fin || *abort_flag)) break;
+      if (named_bar_or(1 + g, 128, !got || fin || *abort_flag)) {
+        if (gt == 0) bulk_wait_all();  // copies out of shared memory end before the CTA does
+        break;
+      }
       const int L = meta[MT_L];
       const int si = meta[MT_I];
       const int pos = meta[MT_POS];
       const int hh = meta[MT_H];
       if (gt == 0) {
         // this chunk's ring slot must have been copied out by its state CTA
-        if (pos + 1 - NRING > 0)
-          spin_geq(gflags + F_REC0 + si * F_REC_STRIDE + F_CONSUMED, static_cast<uint32_t>(pos + 1 - NRING),
+        if (pos + 1 - p.nring > 0)
+          spin_geq(gflags + F_REC0 + si * F_REC_STRIDE + F_CONSUMED, static_cast<uint32_t>(pos + 1 - p.nring),
                    gflags + F_ABORT, abort_flag);
       }
       const int64_t t0 = static_cast<int64_t>((static_cast<uint64_t>(static_cast<uint32_t>(meta[MT_T0HI])) << 32) |
                                               static_cast<uint32_t>(meta[MT_T0LO]));
-      uint8_t* slot = p.ring + (static_cast<size_t>(si) * NRING + (pos % NRING)) * SLOT;
+      uint8_t* slot = p.ring + (static_cast<size_t>(si) * p.nring + (pos % p.nring)) * SLOT;
       // beta of this chunk (rows >= L are zero); the load overlaps the cumsum
       // MMA, and the group owns its copy (the load warp moves on to the next
       // chunk as soon as the raw tiles are released)
@@ -549,6 +562,12 @@ struct Tf {
         vec[128 + gt] = ex2_approx(gl);
       }
       bar();
+      // q_r . k_r over this thread's channel half, in fp32 from the raw bf16
+      // inputs: the diagonal of P, where the decay factors cancel exactly.  The
+      // bf16-rounded scaled operands would lose it to cancellation when q_r and
+      // k_r are nearly orthogonal (it is the whole output of a token that
+      // starts from a zero state).
+      float pdiag = 0.f;
       if (!slow) {
 #pragma unroll
         for (int jj = 0; jj < 8; ++jj) {
@@ -567,8 +586,8 @@ struct Tf {
           uint32_t ka[4], qa[4], kb[4], kt[4];
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            const int c = c0 + 2 * u;
             const float2 kx = bf2f(kk4[u]), qx = bf2f(qq4[u]);
+            pdiag = fmaf(qx.x, kx.x, fmaf(qx.y, kx.y, pdiag));
             const float rf0 = rf8[2 * u], rf1 = rf8[2 * u + 1];
             const float x0 = g2[8 * jj + 2 * u], x1 = g2[8 * jj + 2 * u + 1];
             const float e10 = ex2_approx(x0 - rf0), e11 = ex2_approx(x1 - rf1);
@@ -585,6 +604,11 @@ struct Tf {
           // Kt replaces the raw k chunk this thread just read (ring layout)
           sts128(gb + LY::G_RK + ch * 8192 + sw128(r, jj), make_uint4(kt[0], kt[1], kt[2], kt[3]));
         }
+        // the first channel half hands its partial to the thread of the second
+        // half that writes row r of P (same r), through the upper half of the
+        // log-decay tile: dead since the cumsum MMA completed, not reloaded
+        // before this chunk's raw tiles are released, and not under P
+        if (ch == 0) reinterpret_cast<float*>(gb + LY::G_RL + 8192)[r] = pdiag;
       } else {
         // ---- exact path: A and P term by term from g (fp32, in the KQ area) ------
         float* G = reinterpret_cast<float*>(gb + LY::G_KQ);
@@ -685,14 +709,17 @@ struct Tf {
             *reinterpret_cast<float4*>(Af + swzA(ar, 4 * s4)) = w;
           }
         } else {
-          const int rp = 32 * (q - 2) + lane;
+          const int rp = 32 * (q - 2) + lane;  // == r of this thread (channel half 1)
+          const float dg = pdiag + reinterpret_cast<const float*>(gb + LY::G_RL + 8192)[rp];
 #pragma unroll
           for (int jj = 0; jj < 8; ++jj) {
             uint32_t pk[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
               const int s0 = 8 * jj + 2 * u;
-              pk[u] = pack_bf16(s0 <= rp ? x[s0] : 0.f, s0 + 1 <= rp ? x[s0 + 1] : 0.f);
+              const float p0 = s0 < rp ? x[s0] : (s0 == rp ? dg : 0.f);
+              const float p1 = s0 + 1 < rp ? x[s0 + 1] : (s0 + 1 == rp ? dg : 0.f);
+              pk[u] = pack_bf16(p0, p1);
             }
             sts128(gb + LY::G_RL + sw128(rp, jj), make_uint4(pk[0], pk[1], pk[2], pk[3]));
           }
@@ -928,14 +955,14 @@ __device__ __forceinline__ void state_load_loop(uint8_t* smem, const Maps& maps,
         ok = false;
         break;
       }
-      if (!spin_geq(ready + (pos % NRING), static_cast<uint32_t>(pos + 1), gflags + F_ABORT, abort_flag)) {
+      if (!spin_geq(ready + (pos % p.nring), static_cast<uint32_t>(pos + 1), gflags + F_ABORT, abort_flag)) {
         ok = false;
         break;
       }
       fence_proxy_async_global();
       const int64_t t0 = w.sb + static_cast<int64_t>(j) * C;
       mbar_arrive_expect_tx(&bars[BS_SLOT_FULL + s], SLOT + 16384);
-      const uint8_t* src = p.ring + (static_cast<size_t>(i) * NRING + (pos % NRING)) * SLOT;
+      const uint8_t* src = p.ring + (static_cast<size_t>(i) * p.nring + (pos % p.nring)) * SLOT;
       uint8_t* dst = smem + ST_SLOT + s * SLOT;
       bulk_g2s(dst, src, 32768, &bars[BS_SLOT_FULL + s]);
       bulk_g2s(dst + 32768, src + 32768, SLOT - 32768, &bars[BS_SLOT_FULL + s]);
@@ -992,7 +1019,10 @@ __device__ __forceinline__ void state_mma_loop(uint32_t sbase, uint32_t tmem, co
       for (int kk = 0; kk < 8; ++kk)
         mma_bf16_ss(tmem + TS_U, make_sdesc_sw128(sbase + ST_S + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
                     make_sdesc_sw128(slot + R_WT + kk * 2048, 8192, 1024), id_us, 1);
-      mma_commit(&bars[BS_U_FULL]);
+#ifdef KDA_TEST_HOOKS
+      if (!(g_test_skip_commit != 0 && blockIdx.x == 0 && pos == 0))
+#endif
+        mma_commit(&bars[BS_U_FULL]);
       // O = Qa S'  (M = 64 rows r, N = 128 values v; buffer b, free once
       // position pos-2 was read out; S' is the K-major B operand [v][c])
       if (pos >= 2 && !mbar_wait(&bars[BS_O_FREE + b], ((pos - 2) >> 1) & 1, abort_flag)) { ok = false; break; }
@@ -1092,10 +1122,12 @@ __device__ __forceinline__ void state_warps_loop(uint8_t* smem, uint32_t tmem, c
   StateWalk w{i - p.R, 0, 0, 0};
   while (ok && w.next(p)) {
     const int n = w.ci / p.H, h = w.ci % p.H;
-    const size_t sidx = (static_cast<size_t>(n) * p.H + h) * D * D;
-    if (p.S0) {
+    bool rd, wr;
+    const int row = state_row(p.st, n, &rd, &wr);
+    const size_t sidx = (static_cast<size_t>(row < 0 ? 0 : row) * p.H + h) * D * D;
+    if (rd) {
 #pragma unroll
-      for (int u = 0; u < 64; ++u) S[u] = p.S0[sidx + static_cast<size_t>(64 * hf + u) * D + v];
+      for (int u = 0; u < 64; ++u) S[u] = p.st.S0[sidx + static_cast<size_t>(64 * hf + u) * D + v];
     } else {
 #pragma unroll
       for (int u = 0; u < 64; ++u) S[u] = 0.f;
@@ -1169,9 +1201,9 @@ __device__ __forceinline__ void state_warps_loop(uint8_t* smem, uint32_t tmem, c
       have_prev = true;
     }
     if (!ok) break;
-    if (p.S_T) {
+    if (wr) {
 #pragma unroll
-      for (int u = 0; u < 64; ++u) p.S_T[sidx + static_cast<size_t>(64 * hf + u) * D + v] = S[u];
+      for (int u = 0; u < 64; ++u) p.st.S_T[sidx + static_cast<size_t>(64 * hf + u) * D + v] = S[u];
     }
   }
   if (ok && have_prev) o_pass(pos - 1);

@@ -16,7 +16,11 @@ namespace kda {
 // kda_check_device_error().
 __device__ int g_device_error = 0;
 
+#ifdef KDA_TEST_HOOKS
+constexpr long long kWaitCycles = 200000000LL;  // ~0.1 s: the test build makes waits run out quickly
+#else
 constexpr long long kWaitCycles = 4000000000LL;  // ~2 s at 2 GHz
+#endif
 
 __device__ __forceinline__ void record_error(int code) { atomicCAS(&g_device_error, 0, code); }
 

@@ -17,6 +17,7 @@
 #pragma once
 
 #include "kda_ptx.cuh"
+#include "kda_state_io.cuh"
 
 namespace kda {
 
@@ -145,16 +146,28 @@ __device__ __forceinline__ void recurrent_run(int64_t t0, int64_t t1, int h, int
   }
 }
 
-// Decode: blockIdx.x = n * H + h; token n of the [N, H, d] inputs.
+// Decode: blockIdx.x = n * H + h; token n of the [N, H, d] inputs.  The state
+// of sequence n is row n of S, or pool slot slots[n] when slots is given; a
+// negative slot has no cached state: the token runs from a zero state and the
+// new state is dropped.
 template <int DK, int DV, typename TIO, typename TG>
 __global__ void __launch_bounds__(kRecThreads, 2)
     kda_decode_kernel(int H, const TIO* __restrict__ q, const TIO* __restrict__ k, const TIO* __restrict__ v,
-                      const TG* __restrict__ la, const TG* __restrict__ beta, float* S, TIO* __restrict__ o) {
+                      const TG* __restrict__ la, const TG* __restrict__ beta, float* S, TIO* __restrict__ o,
+                      const int32_t* __restrict__ slots, int num_slots) {
   __shared__ __align__(16) RecSmem<DK, DV> sm;
   const int nh = blockIdx.x;
   const int n = nh / H, h = nh % H;
-  float* Snh = S + static_cast<int64_t>(nh) * DK * DV;
-  recurrent_run<DK, DV, TIO, TG, true>(n, n + 1, h, H, q, k, v, la, beta, Snh, Snh, o, sm);
+  StateIO io;
+  io.S0 = S;
+  io.S_T = S;
+  io.slots = slots;
+  io.num_slots = num_slots;
+  bool rd, wr;
+  const int row = state_row(io, n, &rd, &wr);
+  float* Snh = S + (static_cast<int64_t>(row < 0 ? 0 : row) * H + h) * DK * DV;
+  recurrent_run<DK, DV, TIO, TG, true>(n, n + 1, h, H, q, k, v, la, beta, rd ? Snh : nullptr, wr ? Snh : nullptr, o,
+                                       sm);
 }
 
 // Prefill on CUDA cores: blockIdx.x = h, blockIdx.y = sequence n.
@@ -162,7 +175,7 @@ template <int DK, int DV, typename TIO, typename TG>
 __global__ void __launch_bounds__(kRecThreads, 2)
     kda_recurrent_fwd_kernel(int H, int T, const int32_t* __restrict__ cu_seqlens, const TIO* __restrict__ q,
                              const TIO* __restrict__ k, const TIO* __restrict__ v, const TG* __restrict__ la,
-                             const TG* __restrict__ beta, const float* S0, TIO* __restrict__ o, float* S_T) {
+                             const TG* __restrict__ beta, StateIO io, TIO* __restrict__ o) {
   __shared__ __align__(16) RecSmem<DK, DV> sm;
   const int h = blockIdx.x, n = blockIdx.y;
   int64_t t0, t1;
@@ -173,9 +186,11 @@ __global__ void __launch_bounds__(kRecThreads, 2)
     t0 = static_cast<int64_t>(n) * T;
     t1 = t0 + T;
   }
-  const int64_t off = (static_cast<int64_t>(n) * H + h) * DK * DV;
-  recurrent_run<DK, DV, TIO, TG, false>(t0, t1, h, H, q, k, v, la, beta, S0 ? S0 + off : nullptr,
-                                        S_T ? S_T + off : nullptr, o, sm);
+  bool rd, wr;
+  const int row = state_row(io, n, &rd, &wr);
+  const int64_t off = (static_cast<int64_t>(row < 0 ? 0 : row) * H + h) * DK * DV;
+  recurrent_run<DK, DV, TIO, TG, false>(t0, t1, h, H, q, k, v, la, beta, rd ? io.S0 + off : nullptr,
+                                        wr ? io.S_T + off : nullptr, o, sm);
 }
 
 }  // namespace kda

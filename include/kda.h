@@ -32,8 +32,8 @@
  *     failing check returns an error status and launches nothing.
  *   - The library never aborts, asserts, traps or prints.
  *   - Alignment (KDA_ERR_ALIGN otherwise): S0, S_T, S and the workspace
- *     16 bytes; q, k, v, o and log_alpha 4 bytes; beta and cu_seqlens their
- *     element size.
+ *     16 bytes; q, k, v, o and log_alpha 4 bytes (16 bytes on the tensor-core
+ *     path, see kda_chunk_fwd); beta and cu_seqlens their element size.
  *   - Contiguous layouts (token-major, head next, channel innermost):
  *       q, k, log_alpha : [B, T, H, dk]        v, o : [B, T, H, dv]
  *       beta            : [B, T, H]
@@ -52,7 +52,7 @@
 extern "C" {
 #endif
 
-#define KDA_ABI_VERSION 1
+#define KDA_ABI_VERSION 3
 
 typedef enum {
   KDA_OK = 0,
@@ -76,7 +76,7 @@ typedef struct kda_shape {
   int32_t T;          /* tokens per batch row; packed total with cu_seqlens  */
   int32_t H;          /* heads                                               */
   int32_t dk, dv;     /* key / value head dimensions: 64 or 128 each         */
-  int32_t chunk;      /* chunk length C of the chunkwise form: 16, 32 or 64  */
+  int32_t chunk;      /* chunk length C of the chunkwise form: must be 64    */
   int32_t n_seqs;     /* N = number of packed sequences (with cu_seqlens)    */
   int32_t io_dtype;   /* kda_dtype of q, k, v and o                          */
   int32_t gate_dtype; /* kda_dtype of log_alpha and beta                     */
@@ -86,26 +86,29 @@ typedef struct kda_shape {
 /* Copy cu_seqlens to the host and check it before launching.  This
  * synchronises `stream`; without the flag cu_seqlens is trusted. */
 #define KDA_FLAG_VALIDATE_CU_SEQLENS 0x1u
-/* Run the tensor-core chunk path as two kernels (a fully parallel prep over
- * every (chunk, head) writing MMA-ready operands to the workspace, then the
- * inter-chunk recurrence) instead of the default pipelined kernel. */
-#define KDA_FLAG_PATH_TWO_PASS 0x2u
-/* Tuning of the pipelined tensor-core path (0 = automatic):
- * KDA_FLAG_STATE_CTAS(n) fixes the number of state CTAs (each walks whole
- * (sequence, head) chains), KDA_FLAG_GRID_CTAS(n) caps the number of CTAs of
- * the launch (at most one per SM).  Values are clamped to what the problem and
- * the device allow.  kda_chunk_fwd_workspace_size() depends on both. */
+/* Run the token-by-token CUDA-core recurrence (fp32, no chunking) even where
+ * the tensor-core path applies; fp32 io and dk or dv = 64 always take it.  A
+ * reference path for validation, not a fast one. */
+#define KDA_FLAG_PATH_RECURRENT 0x4u
+/* Tuning of the tensor-core path (0 = automatic): KDA_FLAG_STATE_CTAS(n)
+ * fixes the number of state CTAs (each walks whole (sequence, head) chains),
+ * KDA_FLAG_GRID_CTAS(n) caps the number of CTAs of the launch (at most one per
+ * SM).  Values are clamped to what the problem and the device allow.
+ * kda_chunk_fwd_workspace_size() depends on both. */
 #define KDA_FLAG_STATE_CTAS(n) ((((uint32_t)(n)) & 0xFFu) << 8)
 #define KDA_FLAG_GRID_CTAS(n) ((((uint32_t)(n)) & 0xFFu) << 16)
 
 /*
- * kda_chunk_fwd_workspace_size -- bytes of device workspace kda_chunk_fwd
- * needs for `shape` on the CURRENT device.  0 on the CUDA-core paths.  On the
- * tensor-core path: a ring of 8 operand slots of 66,560 bytes per state CTA
- * plus a few KB of counters (at most ~40 MB on a 148-SM B200, independent of
- * the sequence lengths); with KDA_FLAG_PATH_TWO_PASS one 82,432-byte slot per
- * (chunk, head).  Returns 0 for shapes the library rejects; kda_chunk_fwd then
- * reports the reason.
+ * kda_chunk_fwd_workspace_size -- preferred bytes of device workspace for
+ * kda_chunk_fwd with `shape` on the CURRENT device.  0 on the CUDA-core path.
+ * On the tensor-core path the workspace holds a few KB of counters and an
+ * operand ring of up to 16 slots of 66,560 bytes for each of R "state" CTAs
+ * (R is chosen per call from the number of (sequence, head) pairs and the SM
+ * count, at most one less than the SM count): at most ~160 MB on a 148-SM
+ * B200, typically 20-80 MB, independent of the sequence lengths.  A smaller
+ * workspace also works, down to a 2-slot ring, with a shallower and slower
+ * pipeline; below that kda_chunk_fwd returns KDA_ERR_WORKSPACE.  Returns 0
+ * for shapes the library rejects; kda_chunk_fwd then reports the reason.
  */
 size_t kda_chunk_fwd_workspace_size(const kda_shape* shape);
 
@@ -120,22 +123,22 @@ size_t kda_chunk_fwd_workspace_size(const kda_shape* shape);
  *   cu_seqlens  NULL for a dense batch, else N+1 int32 offsets (B == 1).
  *   o           output [B, T, H, dv] in io_dtype; must not alias an input.
  *   S_T         final states [N, H, dk, dv] fp32, or NULL; may alias S0.
- *   workspace   device scratch of at least kda_chunk_fwd_workspace_size()
- *               bytes (NULL allowed when that size is 0); contents on entry
- *               are ignored and on exit undefined.
+ *   workspace   device scratch (see kda_chunk_fwd_workspace_size; NULL
+ *               allowed when that size is 0); contents on entry are ignored
+ *               and on exit undefined.
  *
- * Paths: bf16 io with dk = dv = 128 and chunk = 64 runs on the tcgen05
- * tensor cores (fp32 state, bf16 operands, fp32 accumulation).  By default one
- * cooperative launch with one CTA per SM: "state" CTAs each carry whole
- * (sequence, head) chains through their chunks, "transform" CTAs compute the
- * state-independent per-chunk operands in parallel and hand them over through
- * a ring in the workspace.  q, k, v and log_alpha must then be 16-byte aligned
- * (they are read by TMA).  With KDA_FLAG_PATH_TWO_PASS a prep kernel plus a
- * recurrence kernel through a larger workspace.  Every other supported shape,
- * and all fp32 io, runs the fp32 CUDA-core recurrent kernel (token by token,
- * which keeps fp32 inputs within the 1e-4 tolerance).  Sequences of length 0
- * copy S0 to S_T.  The call must not overlap another use of the same
- * workspace on the GPU.
+ * Paths: bf16 io with dk = dv = 128 runs on the tcgen05 tensor cores (fp32
+ * state, bf16 operands, fp32 accumulation), one cooperative launch with one
+ * CTA per SM: "state" CTAs each carry whole (sequence, head) chains through
+ * their chunks, "transform" CTAs compute the state-independent per-chunk
+ * operands in parallel and hand them over through a ring in the workspace.
+ * q, k, v, log_alpha and o must then be 16-byte aligned (TMA reads, 16-byte
+ * row stores).  fp32 io, dk or dv = 64, and KDA_FLAG_PATH_RECURRENT run the
+ * fp32 token-by-token CUDA-core recurrence instead (it keeps fp32 inputs
+ * within the 1e-4 tolerance; it is latency-bound, three barriers per token).
+ * The chunk length is 64 on every path.  Sequences of length 0 copy S0 to
+ * S_T.  The call must not overlap another use of the same workspace on the
+ * GPU.
  */
 kda_status kda_chunk_fwd(const kda_shape* shape, const void* q, const void* k, const void* v,
                          const void* log_alpha, const void* beta, const float* S0,
@@ -157,11 +160,11 @@ kda_status kda_chunk_fwd(const kda_shape* shape, const void* q, const void* k, c
  *
  *   - The array holds KDA_NOALLOC_SCRATCH_BYTES (64 MiB).  Every GPU that
  *     loads the library reserves it until the process exits.
- *   - A shape whose kda_chunk_fwd_workspace_size() exceeds that is rejected
- *     with KDA_ERR_WORKSPACE before anything is launched.  The default
- *     tensor-core path needs at most ~40 MB on a 148-SM B200 whatever the
- *     sequence lengths; KDA_FLAG_PATH_TWO_PASS needs one 82,432-byte slot per
- *     (chunk, head) and fits up to 814 of them.
+ *   - The tensor-core path sizes its operand ring to what fits the array (2
+ *     to 16 slots per state CTA).  A shape that cannot fit even the 2-slot
+ *     ring is rejected with KDA_ERR_WORKSPACE before anything is launched; on
+ *     a 148-SM B200 that ring needs at most ~20 MB, so no valid shape is
+ *     rejected there.  The CUDA-core path needs no scratch.
  *   - Every call looks up the array's device address (cudaGetSymbolAddress)
  *     on the current device; the lookup allocates nothing.  The first call on
  *     a device may load the library's device code there, so make that first
@@ -192,6 +195,46 @@ kda_status kda_chunk_fwd_noalloc(const kda_shape* shape, const void* q, const vo
 kda_status kda_decode_step(const kda_shape* shape, const void* q, const void* k, const void* v,
                            const void* log_alpha, const void* beta, float* S, void* o,
                            void* stream);
+
+/*
+ * Serving-state variants.  A serving engine keeps the recurrent states of its
+ * live requests in one pool, [num_slots, H, dk, dv] fp32, and hands each
+ * batch an int32 slot index per sequence (continuous batching: the batch is
+ * a permutation of live requests, not a prefix of the pool).  These calls
+ * read and write the states in place in the pool through that index; they
+ * are otherwise kda_chunk_fwd and kda_decode_step.
+ *
+ *   state_pool     [num_slots, H, dk, dv] fp32 device array, 16-byte aligned;
+ *                  read and overwritten in place.
+ *   num_slots      rows of the pool (> 0).
+ *   state_slots    int32 device array with one entry per sequence (N for the
+ *                  prefill, B for the decode step).  slot >= 0: the state of
+ *                  that sequence lives in that pool row.  slot < 0: padding,
+ *                  the sequence has no cached state: it runs from a zero state
+ *                  and its final state is dropped (its output is still
+ *                  written).  slot >= num_slots is refused on the device: that
+ *                  sequence is treated as padding and the call records
+ *                  KDA_ERR_ARGUMENT for kda_check_device_error.
+ *                  Non-negative slots of one call must be distinct (two
+ *                  sequences writing one row give an undefined state).
+ *   has_initial_state  (prefill only) uint8 device array, one per sequence:
+ *                  0 = start from zeros (a new request; the pool row's old
+ *                  contents are ignored), else resume from the state in the
+ *                  pool (a prompt continued after a cached prefix, or a
+ *                  chunked prefill).  NULL = resume for every sequence.
+ *
+ * The other arguments, the paths and the errors are those of kda_chunk_fwd
+ * (workspace: kda_chunk_fwd_workspace_size) and kda_decode_step.
+ */
+kda_status kda_chunk_fwd_slots(const kda_shape* shape, const void* q, const void* k, const void* v,
+                               const void* log_alpha, const void* beta, float* state_pool, int32_t num_slots,
+                               const int32_t* state_slots, const uint8_t* has_initial_state,
+                               const int32_t* cu_seqlens, void* o, void* workspace, size_t workspace_bytes,
+                               void* stream);
+
+kda_status kda_decode_step_slots(const kda_shape* shape, const void* q, const void* k, const void* v,
+                                 const void* log_alpha, const void* beta, float* state_pool, int32_t num_slots,
+                                 const int32_t* state_slots, void* o, void* stream);
 
 /*
  * kda_check_device_error -- synchronises `stream`, then returns and clears

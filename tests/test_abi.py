@@ -30,7 +30,7 @@ def test_library_loads_and_exports_every_declared_symbol():
     lib = kda.load_library()
     for name in declared_functions():
         assert hasattr(lib, name), name
-    assert kda.kda_abi_version() == 1
+    assert kda.kda_abi_version() == 3
 
 
 def test_status_strings():
@@ -68,7 +68,8 @@ def test_null_shape():
 
 @pytest.mark.parametrize("field,value,status", [
     ("io_dtype", 7, -3), ("gate_dtype", -1, -3), ("B", 0, -2), ("H", 0, -2), ("T", -1, -2),
-    ("dk", 96, -5), ("dv", 32, -5), ("chunk", 48, -5), ("flags", 0x80, -10),
+    ("dk", 96, -5), ("dv", 32, -5), ("chunk", 48, -5), ("chunk", 32, -5), ("chunk", 16, -5),
+    ("flags", 0x80, -10), ("flags", 0x2, -10),
 ])
 def test_bad_shape_fields(field, value, status):
     assert call_fwd(tc_shape(**{field: value})) == status
@@ -82,20 +83,16 @@ def test_null_inputs_and_misalignment():
     assert call_fwd(tc_shape(), {"S0": FAKE + 8}) == -4
 
 
-def test_workspace_required_for_two_pass_path():
-    s = tc_shape(B=2, T=200, flags=kda.KDA_FLAG_PATH_TWO_PASS)
-    need = kda.kda_chunk_fwd_workspace_size(s)
-    # (floor(400/64) + 2 sequences) chunks x 2 heads x one 82,432-byte slot
-    assert need == (400 // 64 + 2) * 2 * 82432
-    assert call_fwd(s) == -6
-    assert call_fwd(s, ws=FAKE, ws_bytes=need - 16) == -6
-    assert call_fwd(s, ws=FAKE + 4, ws_bytes=need) == -4
+def test_workspace_required_on_tensor_core_path():
+    # without a workspace the call is refused (KDA_ERR_WORKSPACE), or, on a
+    # machine without a GPU, fails while sizing the launch (KDA_ERR_CUDA)
+    assert call_fwd(tc_shape(B=2, T=200)) in (-6, -7)
 
 
 def test_cuda_core_paths_need_no_workspace():
     assert kda.kda_chunk_fwd_workspace_size(tc_shape(io_dtype=0)) == 0
     assert kda.kda_chunk_fwd_workspace_size(tc_shape(dk=64, dv=64)) == 0
-    assert kda.kda_chunk_fwd_workspace_size(tc_shape(chunk=32)) == 0
+    assert kda.kda_chunk_fwd_workspace_size(tc_shape(flags=kda.KDA_FLAG_PATH_RECURRENT)) == 0
 
 
 def test_tuning_flags_are_accepted_and_encoded():
@@ -113,9 +110,9 @@ def test_pipelined_path_workspace_is_bounded_by_the_sm_count():
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     small = kda.kda_chunk_fwd_workspace_size(tc_shape())
     big = kda.kda_chunk_fwd_workspace_size(tc_shape(B=1, T=1 << 20, H=64))
-    assert 0 < small <= big <= sms * 8 * 66560 + 65536
+    assert 0 < small <= big <= sms * 16 * 66560 + 65536
     capped = kda.kda_chunk_fwd_workspace_size(tc_shape(H=64, flags=kda.tuning_flags(3, 0)))
-    assert capped < 4 * 8 * 66560 + 65536
+    assert capped < 4 * 16 * 66560 + 65536
 
 
 def test_packed_requires_single_batch_row():
@@ -127,6 +124,39 @@ def test_decode_rejects_multi_token():
     s = kda.make_shape(4, 2, 2, 128, 128)
     args = [ctypes.c_void_p(FAKE)] * 7
     assert lib.kda_decode_step(ctypes.byref(s), *args, None) == -2
+
+
+def call_fwd_slots(shape, pool=FAKE, num_slots=4, slots=FAKE, has_init=None, cu=None):
+    lib = kda.load_library()
+    vp = lambda x: None if x is None else ctypes.c_void_p(x)
+    f = vp(FAKE)
+    return lib.kda_chunk_fwd_slots(ctypes.byref(shape), f, f, f, f, f, vp(pool), num_slots, vp(slots),
+                                   vp(has_init), vp(cu), f, None, 0, None)
+
+
+def test_slot_prefill_host_validation():
+    assert call_fwd_slots(tc_shape(), pool=None) == -1
+    assert call_fwd_slots(tc_shape(), slots=None) == -1
+    assert call_fwd_slots(tc_shape(), num_slots=0) == -2
+    assert call_fwd_slots(tc_shape(), slots=FAKE + 2) == -4
+    assert call_fwd_slots(tc_shape(), pool=FAKE + 8) == -4
+    assert call_fwd_slots(tc_shape(chunk=32)) == -5
+    # the CUDA-core path needs no workspace: it gets as far as the launch
+    # (which fails on a machine without a GPU)
+    assert call_fwd_slots(tc_shape(B=2, T=200)) in (-6, -7)
+
+
+def test_slot_decode_host_validation():
+    lib = kda.load_library()
+    f = ctypes.c_void_p(FAKE)
+    call = lambda shape, pool, n, slots: lib.kda_decode_step_slots(ctypes.byref(shape), f, f, f, f, f, pool, n,
+                                                                   slots, f, None)
+    s1 = kda.make_shape(4, 1, 2, 128, 128)
+    assert call(s1, f, 4, None) == -1
+    assert call(s1, None, 4, f) == -1
+    assert call(s1, f, 0, f) == -2
+    assert call(kda.make_shape(4, 2, 2, 128, 128), f, 4, f) == -2
+    assert call(s1, f, 4, ctypes.c_void_p(FAKE + 2)) == -4
 
 
 def test_python_binding_refuses_cpu_tensors():

@@ -60,10 +60,10 @@ def _check_fwd(x, tol, o=None, S=None, seq_slices=None):
     return err_o, err_S
 
 
-def _run(x, chunk=64, two_pass=False):
+def _run(x, **kw):
     xd = _dev(x)
     o, S = kda.kda_chunk_fwd(xd["q"], xd["k"], xd["v"], xd["log_alpha"], xd["beta"], xd["S0"],
-                             xd["cu_seqlens"], chunk=chunk, two_pass=two_pass)
+                             xd["cu_seqlens"], **kw)
     assert kda.kda_check_device_error() == 0
     return o, S
 
@@ -121,73 +121,77 @@ def test_fp32_ragged_varlen(d):
 
 
 # ---------------------------------------------------------------- tensor-core path
-@pytest.mark.parametrize("two_pass", [False, True], ids=["fused", "two_pass"])
-def test_tc_small_batched_ragged_tail(two_pass):
+def test_tc_small_batched_ragged_tail():
     """B=2, T=200 (three full chunks and a ragged tail), H=3, d=128, bf16."""
     x = gen.make_inputs(2, 200, 3, 128, 128, seed=11)
-    o, S = _run(x, two_pass=two_pass)
+    o, S = _run(x)
     _check_fwd(x, TOL_BF16, o, S)
 
 
-@pytest.mark.parametrize("two_pass", [False, True], ids=["fused", "two_pass"])
-def test_tc_varlen_edges(two_pass):
+def test_tc_varlen_edges():
     """Sequences of length 1, 63, 64, 65, 0, 130 and 200 packed together."""
     lens = [1, 63, 64, 65, 0, 130, 200]
     x = gen.make_inputs(1, sum(lens), 2, 128, 128, seqlens=lens, seed=12)
-    o, S = _run(x, two_pass=two_pass)
+    o, S = _run(x)
     _check_fwd(x, TOL_BF16, o, S)
 
 
-@pytest.mark.parametrize("two_pass", [False, True], ids=["fused", "two_pass"])
-def test_tc_fp32_gates(two_pass):
+def test_tc_fp32_gates():
     x = gen.make_inputs(1, 192, 2, 128, 128, gate_dtype=torch.float32, seed=13)
-    o, S = _run(x, two_pass=two_pass)
+    o, S = _run(x)
     _check_fwd(x, TOL_BF16, o, S)
 
 
-@pytest.mark.parametrize("two_pass", [False, True], ids=["fused", "two_pass"])
-def test_tc_no_initial_state(two_pass):
+def test_tc_no_initial_state():
     x = gen.make_inputs(2, 130, 2, 128, 128, s0="none", seed=14)
-    o, S = _run(x, two_pass=two_pass)
+    o, S = _run(x)
     x["S0"] = None
     _check_fwd(x, TOL_BF16, o, S)
 
 
-@pytest.mark.parametrize("two_pass", [False, True], ids=["fused", "two_pass"])
-def test_tc_strong_decay_takes_exact_path(two_pass):
+def test_tc_zero_state_short_sequences():
+    """Sequences of 1-3 tokens from a zero state: the output of a token is
+    beta (q . k) v plus few other terms, so a nearly orthogonal q, k pair
+    makes each (sequence, head) slice ill-conditioned.  The diagonal of the
+    intra-chunk product must not lose q . k to the rounding of the scaled
+    bf16 operands."""
+    lens = [1] * 24 + [2] * 8 + [3] * 8
+    x = gen.make_inputs(1, sum(lens), 4, 128, 128, seqlens=lens, s0="none", seed=33)
+    o, S = _run(x)
+    _check_fwd(x, TOL_BF16, o, S)
+
+
+def test_tc_strong_decay_takes_exact_path():
     """log_alpha = -5 everywhere: each chunk decays 320 nats, beyond the
     factorised form's range; the exact path must still match."""
     x = gen.make_inputs(1, 160, 2, 128, 128, seed=15)
     x["log_alpha"] = torch.full_like(x["log_alpha"], -5.0)
-    o, S = _run(x, two_pass=two_pass)
+    o, S = _run(x)
     _check_fwd(x, TOL_BF16, o, S)
 
 
-@pytest.mark.parametrize("two_pass", [False, True], ids=["fused", "two_pass"])
-def test_tc_no_decay(two_pass):
+def test_tc_no_decay():
     x = gen.make_inputs(1, 192, 2, 128, 128, gate="zero", seed=16)
-    o, S = _run(x, two_pass=two_pass)
+    o, S = _run(x)
     _check_fwd(x, TOL_BF16, o, S)
 
 
-@pytest.mark.parametrize("two_pass", [False, True], ids=["fused", "two_pass"])
-def test_tc_mixed_fast_and_exact_chunks(two_pass):
+def test_tc_mixed_fast_and_exact_chunks():
     """Half the chunks decay beyond the fast path's span, half do not."""
     x = gen.make_inputs(1, 256, 2, 128, 128, seed=17)
     la = x["log_alpha"].float()
     la[:, 64:128] = -4.0
     la[:, 192:256] = -3.0
     x["log_alpha"] = la.to(torch.bfloat16)
-    o, S = _run(x, two_pass=two_pass)
+    o, S = _run(x)
     _check_fwd(x, TOL_BF16, o, S)
 
 
-@pytest.mark.parametrize("two_pass", [False, True], ids=["fused", "two_pass"])
-def test_tc_prefill_workload_sampled(two_pass):
+def test_tc_prefill_workload_sampled():
     """Prefill workload at full size (B4 H16 T4096 d128); oracle on sampled (b, h)."""
     w = gen.workload("prefill")
     x = gen.workload_inputs(w, device="cuda")
-    o, S = kda.kda_chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["S0"], two_pass=two_pass)
+    o, S = kda.kda_chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["S0"])
     assert kda.kda_check_device_error() == 0
     rng = np.random.default_rng(1)
     for b, h in [(0, 0), (3, 15), (int(rng.integers(4)), int(rng.integers(16)))]:
@@ -199,16 +203,22 @@ def test_tc_prefill_workload_sampled(two_pass):
 
 
 # ---------------------------------------------------------------- properties
-def test_tc_paths_match_cuda_core_path():
-    """Same inputs through the fused and two-pass tensor-core paths and the
-    fp32 recurrent path (chunk=32 selects it): all agree within bf16 error."""
+def test_tc_path_matches_cuda_core_path():
+    """Same inputs through the tensor-core path and the fp32 token-by-token
+    CUDA-core recurrence (KDA_FLAG_PATH_RECURRENT): they agree within bf16
+    error."""
     x = _dev(gen.make_inputs(1, 300, 2, 128, 128, seed=21))
-    o1, S1 = kda.kda_chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["S0"], chunk=64)
-    o2, S2 = kda.kda_chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["S0"], chunk=32)
-    o3, S3 = kda.kda_chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["S0"], two_pass=True)
-    for oo, SS in ((o1, S1), (o3, S3)):
-        assert max_rel_l2_per_slice(oo.float().cpu(), o2.float().cpu(), (0, 2)) < TOL_BF16
-        assert max_rel_l2_per_slice(SS.cpu(), S2.cpu(), (0, 1)) < TOL_BF16
+    o1, S1 = kda.kda_chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["S0"])
+    o2, S2 = kda.kda_chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["S0"], recurrent=True)
+    assert max_rel_l2_per_slice(o1.float().cpu(), o2.float().cpu(), (0, 2)) < TOL_BF16
+    assert max_rel_l2_per_slice(S1.cpu(), S2.cpu(), (0, 1)) < TOL_BF16
+
+
+@pytest.mark.parametrize("lens", [[1, 63, 64, 65, 0, 130, 200], [300]])
+def test_recurrent_path_bf16_matches_oracle(lens):
+    x = gen.make_inputs(1, sum(lens), 2, 128, 128, seqlens=lens, seed=27)
+    o, S = _run(x, recurrent=True)
+    _check_fwd(x, TOL_BF16, o, S)
 
 
 def test_tc_split_resume():

@@ -97,15 +97,39 @@ def test_workspace_bytes_are_written_before_they_are_read():
     assert _rel_slices(S.cpu().numpy(), S_or, (0, 1)) <= TOL_BF16
 
 
-def test_noalloc_rejects_shapes_beyond_its_scratch():
-    """A request larger than the built-in 64 MiB is refused before any launch
-    (host-side check, runs without a GPU): the two-pass path's workspace grows
-    with the number of (chunk, head) pairs."""
+@pytest.mark.gpu
+def test_noalloc_runs_the_deepest_ring_its_array_holds():
+    """147 state CTAs want a 16-slot ring of ~156 MB; the 64 MiB array holds
+    a 6-slot ring, which the call uses; the result matches the workspace
+    entry point given its preferred (16-slot) workspace."""
+    x = gen.make_inputs(1, 64, 148, 128, 128, seed=303)
+    xd = {k: (v.cuda() if v is not None else None) for k, v in x.items()}
+    flags = kda.tuning_flags(147, 0)
+    shape = kda.make_shape(1, 64, 148, 128, 128, 64, 0, kda.KDA_BF16, kda.KDA_BF16, flags)
+    assert kda.kda_chunk_fwd_workspace_size(shape) > kda_noalloc_bytes()
+    o_ref, S_ref = kda.kda_chunk_fwd(xd["q"], xd["k"], xd["v"], xd["log_alpha"], xd["beta"], xd["S0"],
+                                     state_ctas=147)
+    o, S_T = torch.empty_like(o_ref), torch.empty_like(S_ref)
     lib = kda.load_library()
-    shape = kda.make_shape(1, 65536, 16, 128, 128, 64, 0, kda.KDA_BF16, kda.KDA_BF16,
-                           kda.KDA_FLAG_PATH_TWO_PASS)
-    assert kda.kda_chunk_fwd_workspace_size(shape) > 64 * 1024 * 1024
+    p = lambda t: ctypes.c_void_p(t.data_ptr())
+    rc = lib.kda_chunk_fwd_noalloc(ctypes.byref(shape), p(xd["q"]), p(xd["k"]), p(xd["v"]), p(xd["log_alpha"]),
+                                   p(xd["beta"]), p(xd["S0"]), None, p(o), p(S_T),
+                                   ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert rc == 0, kda.kda_status_string(rc)
+    assert kda.kda_check_device_error() == 0
+    assert torch.equal(o, o_ref) and torch.equal(S_T, S_ref)
+
+
+def kda_noalloc_bytes():
+    return 64 * 1024 * 1024
+
+
+def test_noalloc_validates_before_touching_the_device():
+    """Invalid shapes are refused on the host with the documented status,
+    without a GPU."""
+    lib = kda.load_library()
     fake = ctypes.c_void_p(0x10000)
-    rc = lib.kda_chunk_fwd_noalloc(ctypes.byref(shape), fake, fake, fake, fake, fake, None, None, fake, None,
-                                   None)
-    assert rc == -6  # KDA_ERR_WORKSPACE
+    assert lib.kda_chunk_fwd_noalloc(None, fake, fake, fake, fake, fake, None, None, fake, None, None) == -1
+    bad = kda.make_shape(1, 128, 2, 128, 128, 32, 0, kda.KDA_BF16, kda.KDA_BF16)
+    assert lib.kda_chunk_fwd_noalloc(ctypes.byref(bad), fake, fake, fake, fake, fake, None, None, fake, None,
+                                     None) == -5
