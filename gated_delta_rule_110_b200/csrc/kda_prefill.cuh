@@ -591,8 +591,9 @@ struct Tf {
             pdiag = fmaf(qx.x, kx.x, fmaf(qx.y, kx.y, pdiag));
             const float rf0 = rf8[2 * u], rf1 = rf8[2 * u + 1];
             const float x0 = g2[8 * jj + 2 * u], x1 = g2[8 * jj + 2 * u + 1];
-            const float e10 = ex2_approx(x0 - rf0), e11 = ex2_approx(x1 - rf1);
-            const float e20 = ex2_approx(rf0 - x0), e21 = ex2_approx(rf1 - x1);
+            const float d0 = x0 - rf0, d1 = x1 - rf1;
+            const float e10 = ex2_approx(d0), e11 = ex2_approx(d1);
+            const float e20 = ex2_approx(-d0), e21 = ex2_approx(-d1);
             ka[u] = pack_bf16(kx.x * e10, kx.y * e11);
             qa[u] = pack_bf16(qx.x * e10, qx.y * e11);
             const float b0 = kx.x * e20, b1 = kx.y * e21;
@@ -732,12 +733,7 @@ struct Tf {
       if (gt == 0) {
         bulk_s2g_hint(slot + R_PP, gb + LY::G_RL, 8192, l2_policy_evict_last());
         bulk_commit();
-        // the inverse writes T over Qa: every copy out of shared memory must
-        // have read its source; then the raw tiles are free for the next chunk
-        bulk_wait_read<0>();
-        mbar_arrive(&bars[BT_RAW_FREE]);
       }
-      bar();
 
       // ---- C4: T = (I + A)^-1, blocked forward substitution (fp32) ---------------
       invert(sbeta);
@@ -871,10 +867,10 @@ struct Tf {
     const int gt = threadIdx.x - 128 * g;
     const float* Af = amat();
     float* X = reinterpret_cast<float*>(gb + LY::G_TB);  // scratch, [3][16][16]
+    float x[16];
     if (gt < 64) {
       // column jc of T_II: x_i = delta_ij - sum_{m<i} A_II[i][m] x_m, one row at a time
       const int I = gt >> 4, jc = gt & 15;
-      float x[16];
 #pragma unroll
       for (int ii = 0; ii < 16; ++ii) {
         const int ra = 16 * I + ii;
@@ -899,6 +895,17 @@ struct Tf {
         }
         x[ii] = acc0 + acc1;
       }
+    }
+    // T overwrites Qa: the copies out of shared memory (Qa, Kt, P) must have
+    // read their sources first; then the raw tiles are free for the next
+    // chunk.  The wait overlaps the diagonal solves above.
+    if (gt == 0) {
+      bulk_wait_read<0>();
+      mbar_arrive(&bars[BT_RAW_FREE]);
+    }
+    bar();
+    if (gt < 64) {
+      const int I = gt >> 4, jc = gt & 15;
 #pragma unroll
       for (int ii = 0; ii < 16; ++ii) trow(16 * I + ii)[tcol(16 * I + ii, 16 * I + jc)] = x[ii];
     }
