@@ -273,7 +273,7 @@ struct Tf {
       const int k = nfinished;
       if (!mbar_wait(&bars[BT_WT_STAGED], k & 1, abort_flag)) return false;
       uint8_t* pslot = p.ring + (static_cast<size_t>(prev_si) * p.nring + (prev_pos % p.nring)) * SLOT;
-      bulk_s2g_hint(pslot + R_WT, gb + LY::G_KB, 16384, l2_policy_evict_last());
+      bulk_s2g(pslot + R_WT, gb + LY::G_KB, 16384);
       bulk_commit();
       bulk_wait_read<0>();
       mbar_arrive(&bars[BT_WT_READ]);
@@ -352,17 +352,16 @@ struct Tf {
         meta[MT_T0HI] = static_cast<int>(static_cast<uint64_t>(t0) >> 32);
         const int y = static_cast<int>(t0);
         mbar_arrive_expect_tx(&bars[BT_RAW_FULL], 32768 + LY::RL_BYTES);
-        const uint64_t pol = l2_policy_evict_first();  // q, k, log-decay are read once
         for (int hf = 0; hf < 2; ++hf) {
-          tma_load_2d_hint(gb + LY::G_RQ + hf * 8192, &maps.q, h * D + 64 * hf, y, &bars[BT_RAW_FULL], pol);
-          tma_load_2d_hint(gb + LY::G_RK + hf * 8192, &maps.k, h * D + 64 * hf, y, &bars[BT_RAW_FULL], pol);
+          tma_load_2d(gb + LY::G_RQ + hf * 8192, &maps.q, h * D + 64 * hf, y, &bars[BT_RAW_FULL]);
+          tma_load_2d(gb + LY::G_RK + hf * 8192, &maps.k, h * D + 64 * hf, y, &bars[BT_RAW_FULL]);
         }
         if (sizeof(TG) == 2) {
           for (int hf = 0; hf < 2; ++hf)
-            tma_load_2d_hint(gb + LY::G_RL + hf * 8192, &maps.la, h * D + 64 * hf, y, &bars[BT_RAW_FULL], pol);
+            tma_load_2d(gb + LY::G_RL + hf * 8192, &maps.la, h * D + 64 * hf, y, &bars[BT_RAW_FULL]);
         } else {
           for (int qq = 0; qq < 4; ++qq)
-            tma_load_2d_hint(gb + LY::G_RL + qq * 8192, &maps.la, h * D + 32 * qq, y, &bars[BT_RAW_FULL], pol);
+            tma_load_2d(gb + LY::G_RL + qq * 8192, &maps.la, h * D + 32 * qq, y, &bars[BT_RAW_FULL]);
         }
         // while this chunk's tiles are in flight, finish the previous chunk
         if (!finish_prev()) stop = 1;
@@ -675,10 +674,9 @@ struct Tf {
         meta[MT_SLOW] = slow ? 1 : 0;
         mbar_arrive(&bars[BT_AP_GO]);
         // Qa (the lower half of each [Ka; Qa] atom) and Kt go to the ring slot
-        const uint64_t pol = l2_policy_evict_last();  // the ring stays in L2 until its state CTA reads it
-        bulk_s2g_hint(slot + R_QA, gb + LY::G_KQ + 8192, 8192, pol);
-        bulk_s2g_hint(slot + R_QA + 8192, gb + LY::G_KQ + 16384 + 8192, 8192, pol);
-        bulk_s2g_hint(slot + R_KT, gb + LY::G_RK, 16384, pol);
+        bulk_s2g(slot + R_QA, gb + LY::G_KQ + 8192, 8192);
+        bulk_s2g(slot + R_QA + 8192, gb + LY::G_KQ + 16384 + 8192, 8192);
+        bulk_s2g(slot + R_KT, gb + LY::G_RK, 16384);
         bulk_commit();
       }
 
@@ -731,7 +729,7 @@ struct Tf {
       fence_proxy_async_smem();
       bar();
       if (gt == 0) {
-        bulk_s2g_hint(slot + R_PP, gb + LY::G_RL, 8192, l2_policy_evict_last());
+        bulk_s2g(slot + R_PP, gb + LY::G_RL, 8192);
         bulk_commit();
       }
 
@@ -765,7 +763,7 @@ struct Tf {
       bar();
       if (gt == 0) {
         mbar_arrive(&bars[BT_W_GO]);
-        bulk_s2g_hint(slot + R_TB, gb + LY::G_TB, 8192, l2_policy_evict_last());
+        bulk_s2g(slot + R_TB, gb + LY::G_TB, 8192);
         bulk_commit();
       }
 
