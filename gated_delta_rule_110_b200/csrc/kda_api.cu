@@ -201,7 +201,8 @@ kda_status launch_prefill(const kda_shape& s, int64_t N, int64_t Ttot, const voi
   const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   bool ok = kda::make_tma_2d(&maps.q, q, bf, 2, cols, rows, cols * 2, 64, 64) &&
             kda::make_tma_2d(&maps.k, k, bf, 2, cols, rows, cols * 2, 64, 64) &&
-            kda::make_tma_2d(&maps.v, v, bf, 2, cols, rows, cols * 2, 64, 64);
+            kda::make_tma_2d(&maps.v, v, bf, 2, cols, rows, cols * 2, 64, 64) &&
+            kda::make_tma_2d(&maps.o, o, bf, 2, cols, rows, cols * 2, 64, 32);
   if (sizeof(TG) == 2)
     ok = ok && kda::make_tma_2d(&maps.la, la, bf, 2, cols, rows, cols * 2, 64, 64);
   else

@@ -85,13 +85,13 @@ constexpr uint32_t ST_SLOT = 0;                   // 2 ring slots
 constexpr uint32_t ST_V = 2 * SLOT;               // 2 x V tile [r][v] (two 64-value atoms)
 constexpr uint32_t ST_S = ST_V + 2 * 16384;       // S'^T [v][c] bf16, two 64-channel atoms
 constexpr uint32_t ST_U = ST_S + 32768;           // U^T [v][r] bf16
-constexpr uint32_t ST_OX = ST_U + 16384;          // per-warp 16 x 128 B transpose scratch for O (8 x 2 KB)
+constexpr uint32_t ST_OX = ST_U + 16384;          // O staging of the two output warps, 2 x [32 rows][128 v] bf16
 constexpr uint32_t ST_BAR = ST_OX + 16384;
 constexpr uint32_t ST_BYTES = ST_BAR + 256;
 // TMEM columns
 constexpr uint32_t TS_U = 0;     // U^T fp32                       64
 constexpr uint32_t TS_DS = 128;  // dS^T fp32                     128
-constexpr uint32_t TS_O = 256;   // 2 x O [r][v] fp32 (M = 64)   2 x 128
+constexpr uint32_t TS_O = 256;   // 2 x O [r][v] fp32, row r in lane 64 + r   2 x 128
 
 // ---- transform CTA shared memory ------------------------------------------------
 template <typename TG>
@@ -131,7 +131,7 @@ enum {
 };
 // state mbarriers
 enum {
-  BS_SLOT_FULL = 0, BS_SLOT_FREE = 2, BS_S_READY = 4, BS_U_FULL, BS_U_READY, BS_DS_FULL, BS_O_FULL,
+  BS_SLOT_FULL = 0, BS_SLOT_FREE = 2, BS_S_READY = 4, BS_U_FULL, BS_U_READY, BS_DS_FULL, BS_SP_FREE, BS_O_FULL,
   BS_O_FREE = BS_O_FULL + 2, BS_FIN = BS_O_FREE + 2, BS_COUNT
 };
 
@@ -151,6 +151,7 @@ struct Params {
 
 struct Maps {
   CUtensorMap q, k, v, la;
+  CUtensorMap o;  // output, box of 64 values x 32 rows
 };
 
 // --------------------------------------------------------------------------- helpers
@@ -997,11 +998,21 @@ __device__ __forceinline__ void state_load_loop(uint8_t* smem, const Maps& maps,
   }
 }
 
+// The MMAs of one position (slot s = b = position parity), in issue order:
+//   U^T  = V^T Tb^T            (state-independent, first)
+//   U^T += S'^T (-W'^T)        -> U_FULL
+//   dS^T = U^T Kt              -> DS_FULL   (the chain: the next S waits on it)
+//   O    = Qa S'               -> SP_FREE   (S' may be overwritten after it)
+//   O   += P U                 -> O_FULL, SLOT_FREE
+// O is produced off the chain, after dS.  Its products are issued with M = 128
+// and an A operand that starts 64 rows before Qa (resp. P) in shared memory,
+// so that the 64 output rows land in TMEM lanes 64-127, where the two output
+// warps (10 and 11) can read them; lanes 0-63 receive unused products.
 __device__ __forceinline__ void state_mma_loop(uint32_t sbase, uint32_t tmem, const Params& p, uint64_t* bars,
                                                volatile int* abort_flag) {
   constexpr uint32_t id_uv = make_idesc_bf16(128, 64) | IDESC_A_MN;
   constexpr uint32_t id_us = make_idesc_bf16(128, 64) | IDESC_B_MN;
-  constexpr uint32_t id_o = make_idesc_bf16(64, 128);
+  constexpr uint32_t id_o = make_idesc_bf16(128, 128);
   constexpr uint32_t id_ds = make_idesc_bf16(128, 128) | IDESC_B_MN;
   const int i = blockIdx.x;
   int pos = 0;
@@ -1030,15 +1041,6 @@ __device__ __forceinline__ void state_mma_loop(uint32_t sbase, uint32_t tmem, co
       if (!(g_test_skip_commit != 0 && blockIdx.x == 0 && pos == 0))
 #endif
         mma_commit(&bars[BS_U_FULL]);
-      // O = Qa S'  (M = 64 rows r, N = 128 values v; buffer b, free once
-      // position pos-2 was read out; S' is the K-major B operand [v][c])
-      if (pos >= 2 && !mbar_wait(&bars[BS_O_FREE + b], ((pos - 2) >> 1) & 1, abort_flag)) { ok = false; break; }
-      tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        mma_bf16_ss(tmem + TS_O + 128 * b,
-                    make_sdesc_sw128(slot + R_QA + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024),
-                    make_sdesc_sw128(sbase + ST_S + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024), id_o, kk > 0);
       if (!mbar_wait(&bars[BS_U_READY], pos & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
       // dS^T = U^T Kt
@@ -1047,10 +1049,21 @@ __device__ __forceinline__ void state_mma_loop(uint32_t sbase, uint32_t tmem, co
         mma_bf16_ss(tmem + TS_DS, make_sdesc_sw128(sbase + ST_U + kk * 32, 16, 1024),
                     make_sdesc_sw128(slot + R_KT + kk * 2048, 8192, 1024), id_ds, kk > 0);
       mma_commit(&bars[BS_DS_FULL]);
-      // O += P U  (U^T [v][r] is the K-major B operand)
+      // O = Qa S'  (buffer b, free once position pos-2 was read out; S'^T [v][c]
+      // is the K-major B operand; the A operand's rows start 8 KB = 64 rows
+      // before each 64-channel atom of Qa)
+      if (pos >= 2 && !mbar_wait(&bars[BS_O_FREE + b], ((pos - 2) >> 1) & 1, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        mma_bf16_ss(tmem + TS_O + 128 * b,
+                    make_sdesc_sw128(slot + R_QA - 8192 + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024),
+                    make_sdesc_sw128(sbase + ST_S + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024), id_o, kk > 0);
+      mma_commit(&bars[BS_SP_FREE]);
+      // O += P U  (U^T [v][r] is the K-major B operand; the A rows start 64 rows before P)
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        mma_bf16_ss(tmem + TS_O + 128 * b, make_sdesc_sw128(slot + R_PP + kk * 32, 16, 1024),
+        mma_bf16_ss(tmem + TS_O + 128 * b, make_sdesc_sw128(slot + R_PP - 8192 + kk * 32, 16, 1024),
                     make_sdesc_sw128(sbase + ST_U + kk * 32, 16, 1024), id_o, 1);
       mma_commit(&bars[BS_O_FULL + b]);
       mma_commit(&bars[BS_SLOT_FREE + s]);
@@ -1061,6 +1074,70 @@ __device__ __forceinline__ void state_mma_loop(uint32_t sbase, uint32_t tmem, co
   const long long t0 = clock64();
   while (!mbar_try_wait(&bars[BS_FIN], 0) && clock64() - t0 < kWaitCycles) {
   }
+}
+
+// Warps 10 and 11 write O: warp 10 + u holds output rows 32 u + lane of a
+// chunk (TMEM lanes 64 + 32 u + lane), 128 values each.  Each warp stages its
+// 32 x 128 block as bf16 in shared memory and stores it with two tensor
+// stores when all its rows belong to the sequence, else row by row.
+__device__ __forceinline__ void state_output_loop(uint8_t* smem, uint32_t tmem, const Maps& maps, const Params& p,
+                                                  uint64_t* bars, volatile int* abort_flag) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int sub = warp - 10;
+  const int r = 32 * sub + lane;
+  const uint32_t lane_off = static_cast<uint32_t>(64 + 32 * sub) << 16;
+  uint8_t* st = smem + ST_OX + sub * 8192;  // [32 rows][128 v] bf16: two 64-value atoms of 4 KB
+  int pos = 0;
+  bool ok = true;
+  StateWalk w{static_cast<int>(blockIdx.x) - p.R, 0, 0, 0};
+  while (ok && w.next(p)) {
+    const int h = w.ci % p.H;
+    for (int j = 0; j < w.nc; ++j, ++pos) {
+      const int b = pos & 1;
+      const int64_t t0 = w.sb + static_cast<int64_t>(j) * C;
+      const int L = static_cast<int>(w.se - t0 < C ? w.se - t0 : C);
+      if (!mbar_wait_warp(&bars[BS_O_FULL + b], (pos >> 1) & 1, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      // the previous tensor store out of the staging block must have read it
+      if (lane == 0) bulk_wait_read<0>();
+      __syncwarp();
+#pragma unroll 1
+      for (int cb = 0; cb < 4; ++cb) {
+        float x[32];
+        tmem_ld32(tmem + lane_off + TS_O + 128 * b + 32 * cb, x);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j4 = 0; j4 < 4; ++j4) {
+          const int vv = 32 * cb + 8 * j4;
+          sts128(st + (vv >> 6) * 4096 + sw128(lane, (vv & 63) >> 3),
+                 make_uint4(pack_bf16(x[8 * j4], x[8 * j4 + 1]), pack_bf16(x[8 * j4 + 2], x[8 * j4 + 3]),
+                            pack_bf16(x[8 * j4 + 4], x[8 * j4 + 5]), pack_bf16(x[8 * j4 + 6], x[8 * j4 + 7])));
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&bars[BS_O_FREE + b]);
+      if (32 * sub + 32 <= L) {
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&maps.o, h * D, static_cast<int>(t0) + 32 * sub, st);
+          tma_store_2d(&maps.o, h * D + 64, static_cast<int>(t0) + 32 * sub, st + 4096);
+          bulk_commit();
+        }
+      } else {
+        __syncwarp();
+        if (r < L) {
+#pragma unroll
+          for (int c16 = 0; c16 < 16; ++c16)
+            *reinterpret_cast<uint4*>(p.o + ((t0 + r) * p.H + h) * D + 8 * c16) =
+                lds128(st + (c16 >> 3) * 4096 + sw128(lane, c16 & 7));
+        }
+        __syncwarp();
+      }
+    }
+  }
+  // tensor stores of O must be complete before the kernel ends
+  if (lane == 0) bulk_wait_all();
 }
 
 // 8 warps; thread (q = warp & 3, hf = warp >> 2) owns value column v = 32 q + lane
@@ -1075,57 +1152,6 @@ __device__ __forceinline__ void state_warps_loop(uint8_t* smem, uint32_t tmem, c
   float S[64];
   int pos = 0;
   bool ok = true;
-  // output of the previous position, read out one step late
-  int prev_L = 0, prev_h = 0;
-  int64_t prev_t0 = 0;
-  bool have_prev = false;
-
-  // O of position pp -> global.  The M = 64 accumulator keeps row r in TMEM
-  // lane 32 (r / 16) + r % 16, so lanes 0-15 of each warp hold one output row
-  // each; a thread stores its 64 values (columns 64 hf ...) with 16-byte
-  // stores, rows past the sequence end skipped.
-  auto o_pass = [&](int pp) -> bool {
-    const int b = pp & 1;
-    if (!mbar_wait_warp(&bars[BS_O_FULL + b], (pp >> 1) & 1, abort_flag)) return false;
-    tc_fence_after();
-    float x[64];
-    {
-      float t[32];
-      tmem_ld32(tmem + lane_off + TS_O + 128 * b + 64 * hf, t);
-      tmem_wait_ld();
-#pragma unroll
-      for (int u = 0; u < 32; ++u) x[u] = t[u];
-      tmem_ld32(tmem + lane_off + TS_O + 128 * b + 64 * hf + 32, t);
-      tmem_wait_ld();
-#pragma unroll
-      for (int u = 0; u < 32; ++u) x[32 + u] = t[u];
-    }
-    tc_fence_before();
-    mbar_arrive(&bars[BS_O_FREE + b]);
-    // lanes 0-15 hold rows 16 q + lane; transpose through the warp's scratch
-    // (128-byte rows, 16-byte chunks XOR-swizzled by row) so that each store
-    // instruction writes 4 whole 128-byte row segments
-    uint8_t* xs = smem + ST_OX + warp * 2048;
-    if (lane < 16) {
-#pragma unroll
-      for (int c8 = 0; c8 < 8; ++c8)
-        sts128(xs + sw128(lane, c8),
-               make_uint4(pack_bf16(x[8 * c8], x[8 * c8 + 1]), pack_bf16(x[8 * c8 + 2], x[8 * c8 + 3]),
-                          pack_bf16(x[8 * c8 + 4], x[8 * c8 + 5]), pack_bf16(x[8 * c8 + 6], x[8 * c8 + 7])));
-    }
-    __syncwarp();
-#pragma unroll
-    for (int k4 = 0; k4 < 4; ++k4) {
-      const int row = 4 * k4 + (lane >> 3), c8 = lane & 7;
-      const int rr = 16 * q + row;
-      const uint4 w = lds128(xs + sw128(row, c8));
-      if (rr < prev_L)
-        *reinterpret_cast<uint4*>(p.o + ((prev_t0 + rr) * p.H + prev_h) * D + 64 * hf + 8 * c8) = w;
-    }
-    __syncwarp();
-    return true;
-  };
-
   StateWalk w{i - p.R, 0, 0, 0};
   while (ok && w.next(p)) {
     const int n = w.ci / p.H, h = w.ci % p.H;
@@ -1143,21 +1169,25 @@ __device__ __forceinline__ void state_warps_loop(uint8_t* smem, uint32_t tmem, c
       const int s = pos & 1;
       const uint8_t* slot = smem + ST_SLOT + s * SLOT;
       if (!mbar_wait_warp(&bars[BS_SLOT_FULL + s], (pos >> 1) & 1, abort_flag)) { ok = false; break; }
-      // S'^T = bf16(sc S^T) -> shared memory (A operand); S <- gamma_C S
+      // S'^T = bf16(sc S^T) -> shared memory (A operand); S <- gamma_C S.  The
+      // previous position's output product must have read the old S' first.
       {
         const float4* sc4 = reinterpret_cast<const float4*>(slot + R_VEC) + 16 * hf;
-        const float4* gc4 = reinterpret_cast<const float4*>(slot + R_VEC) + 32 + 16 * hf;
+        uint32_t pk[32];
 #pragma unroll
-        for (int jj = 0; jj < 8; ++jj) {
-          const float4 a = sc4[2 * jj], b = sc4[2 * jj + 1];
-          const int c = 8 * jj;
-          const uint4 w = make_uint4(pack_bf16(S[c] * a.x, S[c + 1] * a.y), pack_bf16(S[c + 2] * a.z, S[c + 3] * a.w),
-                                     pack_bf16(S[c + 4] * b.x, S[c + 5] * b.y),
-                                     pack_bf16(S[c + 6] * b.z, S[c + 7] * b.w));
-          sts128(smem + ST_S + hf * 16384 + sw128(v, jj), w);
+        for (int u4 = 0; u4 < 16; ++u4) {
+          const float4 a = sc4[u4];
+          pk[2 * u4] = pack_bf16(S[4 * u4] * a.x, S[4 * u4 + 1] * a.y);
+          pk[2 * u4 + 1] = pack_bf16(S[4 * u4 + 2] * a.z, S[4 * u4 + 3] * a.w);
         }
+        if (pos >= 1 && !mbar_wait_warp(&bars[BS_SP_FREE], (pos - 1) & 1, abort_flag)) { ok = false; break; }
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj)
+          sts128(smem + ST_S + hf * 16384 + sw128(v, jj),
+                 make_uint4(pk[4 * jj], pk[4 * jj + 1], pk[4 * jj + 2], pk[4 * jj + 3]));
         fence_proxy_async_smem();
         mbar_arrive(&bars[BS_S_READY]);
+        const float4* gc4 = reinterpret_cast<const float4*>(slot + R_VEC) + 32 + 16 * hf;
 #pragma unroll
         for (int u4 = 0; u4 < 16; ++u4) {
           const float4 gg = gc4[u4];
@@ -1167,7 +1197,6 @@ __device__ __forceinline__ void state_warps_loop(uint8_t* smem, uint32_t tmem, c
           S[4 * u4 + 3] *= gg.w;
         }
       }
-      if (have_prev && !o_pass(pos - 1)) { ok = false; break; }
       // U^T -> bf16 shared memory (A operand)
       if (!mbar_wait_warp(&bars[BS_U_FULL], pos & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
@@ -1201,11 +1230,6 @@ __device__ __forceinline__ void state_warps_loop(uint8_t* smem, uint32_t tmem, c
         for (int u = 0; u < 32; ++u) S[32 + u] += x[u];
       }
       tc_fence_before();
-      const int64_t t0 = w.sb + static_cast<int64_t>(j) * C;
-      prev_t0 = t0;
-      prev_h = h;
-      prev_L = static_cast<int>(w.se - t0 < C ? w.se - t0 : C);
-      have_prev = true;
     }
     if (!ok) break;
     if (wr) {
@@ -1213,7 +1237,6 @@ __device__ __forceinline__ void state_warps_loop(uint8_t* smem, uint32_t tmem, c
       for (int u = 0; u < 64; ++u) p.st.S_T[sidx + static_cast<size_t>(64 * hf + u) * D + v] = S[u];
     }
   }
-  if (ok && have_prev) o_pass(pos - 1);
 }
 
 // ===========================================================================
@@ -1256,8 +1279,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(&bars[BS_DS_FULL], 1);
       mbar_init(&bars[BS_O_FULL + 0], 1);
       mbar_init(&bars[BS_O_FULL + 1], 1);
-      mbar_init(&bars[BS_O_FREE + 0], 256);
-      mbar_init(&bars[BS_O_FREE + 1], 256);
+      mbar_init(&bars[BS_SP_FREE], 1);
+      mbar_init(&bars[BS_O_FREE + 0], 64);
+      mbar_init(&bars[BS_O_FREE + 1], 64);
       mbar_init(&bars[BS_FIN], 1);
     } else {
       for (int g = 0; g < LY::NGROUP; ++g) {
@@ -1301,6 +1325,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       if (lane == 0) state_load_loop(smem, maps, p, bars, abort_flag);
     } else if (warp == 9) {
       if (lane == 0) state_mma_loop(sbase, tmem, p, bars, abort_flag);
+    } else {
+      state_output_loop(smem, tmem, maps, p, bars, abort_flag);
     }
   } else {
     const int g = (warp < 8) ? (warp >> 2) : ((warp - 8) & 1);
