@@ -64,13 +64,19 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kSpan2 = 230.0f;  // largest chunk decay of the factorised path, log2 units
 
 // ---- ring slot: operands of one chunk as the state CTA's MMAs read them ----
-constexpr uint32_t R_TB = 0;       // Tb [r][s] bf16, K-major                     8 KB
-constexpr uint32_t R_WT = 8192;    // -W'^T [c][r] bf16, M/N-major B              16 KB
-constexpr uint32_t R_QA = 24576;   // Qa [r][c] bf16, two 64-channel atoms        16 KB
-constexpr uint32_t R_KT = 40960;   // Kt [r][c] bf16, two 64-channel atoms        16 KB
-constexpr uint32_t R_PP = 57344;   // P [r'][r] bf16, K-major                      8 KB
-constexpr uint32_t R_VEC = 65536;  // sc[128], gC[128] fp32                        1 KB
+// Part A (Tb, -W'^T, the per-channel scales) feeds U and is released once U
+// is formed; part B (Qa, Kt, P) feeds the state update and the output.  The
+// state CTA copies and releases the two parts separately.
+constexpr uint32_t R_TB = 0;       // A: Tb [r][s] bf16, K-major                     8 KB
+constexpr uint32_t R_WT = 8192;    // A: -W'^T [c][r] bf16, M/N-major B              16 KB
+constexpr uint32_t R_VEC = 24576;  // A: sc[128], gC[128] fp32                        1 KB
+constexpr uint32_t R_QA = 25600;   // B: Qa [r][c] bf16, two 64-channel atoms        16 KB
+constexpr uint32_t R_KT = 41984;   // B: Kt [r][c] bf16, two 64-channel atoms        16 KB
+constexpr uint32_t R_PP = 58368;   // B: P [r'][r] bf16, K-major                      8 KB
 constexpr uint32_t SLOT = 66560;
+constexpr uint32_t SLOT_A = R_QA;         // bytes of part A
+constexpr uint32_t SLOT_B = SLOT - R_QA;  // bytes of part B
+static_assert(R_QA % 1024 == 0 && R_KT % 1024 == 0 && R_PP % 1024 == 0 && SLOT % 1024 == 0, "tile alignment");
 
 // ---- global flags (32-bit words) ---------------------------------------------
 constexpr uint32_t F_COUNTER = 0;     // next work item
@@ -81,9 +87,10 @@ constexpr uint32_t F_CONSUMED = 32;
 __host__ __device__ constexpr size_t flag_words(int R) { return F_REC0 + static_cast<size_t>(R) * F_REC_STRIDE; }
 
 // ---- state CTA shared memory --------------------------------------------------
-constexpr uint32_t ST_SLOT = 0;                   // 2 ring slots
-constexpr uint32_t ST_V = 2 * SLOT;               // 2 x V tile [r][v] (two 64-value atoms)
-constexpr uint32_t ST_S = ST_V + 2 * 16384;       // S'^T [v][c] bf16, two 64-channel atoms
+constexpr uint32_t ST_A = 0;                      // 2 x part A (position parity)
+constexpr uint32_t ST_V = ST_A + 2 * SLOT_A;      // 2 x V tile [r][v] (two 64-value atoms)
+constexpr uint32_t ST_B = ST_V + 2 * 16384;       // 2 x part B
+constexpr uint32_t ST_S = ST_B + 2 * SLOT_B;       // S'^T [v][c] bf16, two 64-channel atoms
 constexpr uint32_t ST_U = ST_S + 32768;           // U^T [v][r] bf16
 constexpr uint32_t ST_OX = ST_U + 16384;          // O staging of the two output warps, 2 x [32 rows][128 v] bf16
 constexpr uint32_t ST_BAR = ST_OX + 16384;
@@ -131,7 +138,7 @@ enum {
 };
 // state mbarriers
 enum {
-  BS_SLOT_FULL = 0, BS_SLOT_FREE = 2, BS_S_READY = 4, BS_U_FULL, BS_U_READY, BS_DS_FULL, BS_SP_FREE, BS_O_FULL,
+  BS_A_FULL = 0, BS_A_FREE = 2, BS_B_FULL = 4, BS_B_FREE = 6, BS_S_READY = 8, BS_U_FULL, BS_U_READY, BS_DS_FULL, BS_SP_FREE, BS_O_FULL,
   BS_O_FREE = BS_O_FULL + 2, BS_FIN = BS_O_FREE + 2, BS_COUNT
 };
 
@@ -959,28 +966,30 @@ __device__ __forceinline__ void state_load_loop(uint8_t* smem, const Maps& maps,
     const int h = w.ci % p.H;
     for (int j = 0; j < w.nc; ++j, ++pos) {
       const int s = pos & 1;
-      if (pos >= 2 && !mbar_wait(&bars[BS_SLOT_FREE + s], ((pos - 2) >> 1) & 1, abort_flag)) {
-        ok = false;
-        break;
-      }
+      const uint32_t par = ((pos - 2) >> 1) & 1;
+      // part A and V into buffer s once position pos-2 has finished with them
+      if (pos >= 2 && !mbar_wait(&bars[BS_A_FREE + s], par, abort_flag)) { ok = false; break; }
       if (!spin_geq(ready + (pos % p.nring), static_cast<uint32_t>(pos + 1), gflags + F_ABORT, abort_flag)) {
         ok = false;
         break;
       }
       fence_proxy_async_global();
       const int64_t t0 = w.sb + static_cast<int64_t>(j) * C;
-      mbar_arrive_expect_tx(&bars[BS_SLOT_FULL + s], SLOT + 16384);
       const uint8_t* src = p.ring + (static_cast<size_t>(i) * p.nring + (pos % p.nring)) * SLOT;
-      uint8_t* dst = smem + ST_SLOT + s * SLOT;
-      bulk_g2s(dst, src, 32768, &bars[BS_SLOT_FULL + s]);
-      bulk_g2s(dst + 32768, src + 32768, SLOT - 32768, &bars[BS_SLOT_FULL + s]);
+      mbar_arrive_expect_tx(&bars[BS_A_FULL + s], SLOT_A + 16384);
+      bulk_g2s(smem + ST_A + s * SLOT_A, src, SLOT_A, &bars[BS_A_FULL + s]);
       for (int hf = 0; hf < 2; ++hf)
         tma_load_2d(smem + ST_V + s * 16384 + hf * 8192, &maps.v, h * D + 64 * hf, static_cast<int>(t0),
-                    &bars[BS_SLOT_FULL + s]);
-      // the previous position's copy has landed: its ring slot may be reused
+                    &bars[BS_A_FULL + s]);
+      // part B
+      if (pos >= 2 && !mbar_wait(&bars[BS_B_FREE + s], par, abort_flag)) { ok = false; ++pos; break; }
+      mbar_arrive_expect_tx(&bars[BS_B_FULL + s], SLOT_B);
+      bulk_g2s(smem + ST_B + s * SLOT_B, src + SLOT_A, SLOT_B, &bars[BS_B_FULL + s]);
+      // the previous position's copies have landed: its ring slot may be reused
       if (pos >= 1) {
         const int pp = pos - 1;
-        if (!mbar_wait(&bars[BS_SLOT_FULL + (pp & 1)], (pp >> 1) & 1, abort_flag)) {
+        if (!mbar_wait(&bars[BS_A_FULL + (pp & 1)], (pp >> 1) & 1, abort_flag) ||
+            !mbar_wait(&bars[BS_B_FULL + (pp & 1)], (pp >> 1) & 1, abort_flag)) {
           ok = false;
           ++pos;
           break;
@@ -993,7 +1002,9 @@ __device__ __forceinline__ void state_load_loop(uint8_t* smem, const Maps& maps,
   // drain: copies still landing in shared memory must finish before exit
   for (int pp = pos - 2 < 0 ? 0 : pos - 2; pp < pos; ++pp) {
     const long long t0 = clock64();
-    while (!mbar_try_wait(&bars[BS_SLOT_FULL + (pp & 1)], (pp >> 1) & 1) && clock64() - t0 < kWaitCycles) {
+    while (!mbar_try_wait(&bars[BS_A_FULL + (pp & 1)], (pp >> 1) & 1) && clock64() - t0 < kWaitCycles) {
+    }
+    while (!mbar_try_wait(&bars[BS_B_FULL + (pp & 1)], (pp >> 1) & 1) && clock64() - t0 < kWaitCycles) {
     }
   }
 }
@@ -1003,7 +1014,7 @@ __device__ __forceinline__ void state_load_loop(uint8_t* smem, const Maps& maps,
 //   U^T += S'^T (-W'^T)        -> U_FULL
 //   dS^T = U^T Kt              -> DS_FULL   (the chain: the next S waits on it)
 //   O    = Qa S'               -> SP_FREE   (S' may be overwritten after it)
-//   O   += P U                 -> O_FULL, SLOT_FREE
+//   O   += P U                 -> O_FULL, B_FREE
 // O is produced off the chain, after dS.  Its products are issued with M = 128
 // and an A operand that starts 64 rows before Qa (resp. P) in shared memory,
 // so that the 64 output rows land in TMEM lanes 64-127, where the two output
@@ -1021,33 +1032,38 @@ __device__ __forceinline__ void state_mma_loop(uint32_t sbase, uint32_t tmem, co
   while (ok && w.next(p)) {
     for (int j = 0; j < w.nc; ++j, ++pos) {
       const int s = pos & 1, b = pos & 1;
-      const uint32_t slot = sbase + ST_SLOT + s * SLOT;
+      const uint32_t sa = sbase + ST_A + s * SLOT_A;          // part A of this position
+      const uint32_t sb2 = sbase + ST_B + s * SLOT_B - SLOT_A;  // part B, addressed with ring offsets
       const uint32_t vt = sbase + ST_V + s * 16384;
-      if (!mbar_wait(&bars[BS_SLOT_FULL + s], (pos >> 1) & 1, abort_flag)) { ok = false; break; }
+      if (!mbar_wait(&bars[BS_A_FULL + s], (pos >> 1) & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
       // U^T = V^T Tb^T
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
         mma_bf16_ss(tmem + TS_U, make_sdesc_sw128(vt + kk * 2048, 8192, 1024),
-                    make_sdesc_sw128(slot + R_TB + kk * 32, 16, 1024), id_uv, kk > 0);
+                    make_sdesc_sw128(sa + R_TB + kk * 32, 16, 1024), id_uv, kk > 0);
       if (!mbar_wait(&bars[BS_S_READY], pos & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
       // U^T += S'^T (-W'^T)
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk)
         mma_bf16_ss(tmem + TS_U, make_sdesc_sw128(sbase + ST_S + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                    make_sdesc_sw128(slot + R_WT + kk * 2048, 8192, 1024), id_us, 1);
+                    make_sdesc_sw128(sa + R_WT + kk * 2048, 8192, 1024), id_us, 1);
 #ifdef KDA_TEST_HOOKS
       if (!(g_test_skip_commit != 0 && blockIdx.x == 0 && pos == 0))
 #endif
         mma_commit(&bars[BS_U_FULL]);
       if (!mbar_wait(&bars[BS_U_READY], pos & 1, abort_flag)) { ok = false; break; }
+      // the state warps arrive on U_READY after their last read of the scales:
+      // part A frees once the MMAs issued so far have read it
+      mma_commit(&bars[BS_A_FREE + s]);
+      if (!mbar_wait(&bars[BS_B_FULL + s], (pos >> 1) & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
       // dS^T = U^T Kt
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
         mma_bf16_ss(tmem + TS_DS, make_sdesc_sw128(sbase + ST_U + kk * 32, 16, 1024),
-                    make_sdesc_sw128(slot + R_KT + kk * 2048, 8192, 1024), id_ds, kk > 0);
+                    make_sdesc_sw128(sb2 + R_KT + kk * 2048, 8192, 1024), id_ds, kk > 0);
       mma_commit(&bars[BS_DS_FULL]);
       // O = Qa S'  (buffer b, free once position pos-2 was read out; S'^T [v][c]
       // is the K-major B operand; the A operand's rows start 8 KB = 64 rows
@@ -1057,16 +1073,16 @@ __device__ __forceinline__ void state_mma_loop(uint32_t sbase, uint32_t tmem, co
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk)
         mma_bf16_ss(tmem + TS_O + 128 * b,
-                    make_sdesc_sw128(slot + R_QA - 8192 + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024),
+                    make_sdesc_sw128(sb2 + R_QA - 8192 + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024),
                     make_sdesc_sw128(sbase + ST_S + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024), id_o, kk > 0);
       mma_commit(&bars[BS_SP_FREE]);
       // O += P U  (U^T [v][r] is the K-major B operand; the A rows start 64 rows before P)
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        mma_bf16_ss(tmem + TS_O + 128 * b, make_sdesc_sw128(slot + R_PP - 8192 + kk * 32, 16, 1024),
+        mma_bf16_ss(tmem + TS_O + 128 * b, make_sdesc_sw128(sb2 + R_PP - 8192 + kk * 32, 16, 1024),
                     make_sdesc_sw128(sbase + ST_U + kk * 32, 16, 1024), id_o, 1);
       mma_commit(&bars[BS_O_FULL + b]);
-      mma_commit(&bars[BS_SLOT_FREE + s]);
+      mma_commit(&bars[BS_B_FREE + s]);
     }
     if (!ok) break;
   }
@@ -1167,8 +1183,8 @@ __device__ __forceinline__ void state_warps_loop(uint8_t* smem, uint32_t tmem, c
     }
     for (int j = 0; j < w.nc; ++j, ++pos) {
       const int s = pos & 1;
-      const uint8_t* slot = smem + ST_SLOT + s * SLOT;
-      if (!mbar_wait_warp(&bars[BS_SLOT_FULL + s], (pos >> 1) & 1, abort_flag)) { ok = false; break; }
+      const uint8_t* slot = smem + ST_A + s * SLOT_A;
+      if (!mbar_wait_warp(&bars[BS_A_FULL + s], (pos >> 1) & 1, abort_flag)) { ok = false; break; }
       // S'^T = bf16(sc S^T) -> shared memory (A operand); S <- gamma_C S.  The
       // previous position's output product must have read the old S' first.
       {
@@ -1269,10 +1285,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     *abort_flag = 0;
     if (!is_state) *s_maxlen = 0;
     if (is_state) {
-      mbar_init(&bars[BS_SLOT_FULL + 0], 1);
-      mbar_init(&bars[BS_SLOT_FULL + 1], 1);
-      mbar_init(&bars[BS_SLOT_FREE + 0], 1);
-      mbar_init(&bars[BS_SLOT_FREE + 1], 1);
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(&bars[BS_A_FULL + b], 1);
+        mbar_init(&bars[BS_A_FREE + b], 1);
+        mbar_init(&bars[BS_B_FULL + b], 1);
+        mbar_init(&bars[BS_B_FREE + b], 1);
+      }
       mbar_init(&bars[BS_S_READY], 256);
       mbar_init(&bars[BS_U_FULL], 1);
       mbar_init(&bars[BS_U_READY], 256);
