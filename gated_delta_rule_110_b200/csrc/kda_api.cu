@@ -149,6 +149,8 @@ struct PrefillPlan {
 // kTransformCost times as long per chunk as a state CTA spends on one chunk
 // of its chain.  R minimises the larger of the two times.
 constexpr double kTransformCost = 2.0;
+constexpr size_t kRingL2Bytes = 48u << 20;
+constexpr int kMinPreferredRing = 4;
 
 PrefillPlan plan_prefill(const kda_shape& s, int64_t N, int nsm) {
   PrefillPlan pl;
@@ -178,7 +180,13 @@ PrefillPlan plan_prefill(const kda_shape& s, int64_t N, int nsm) {
   pl.flag_bytes = kda::pipe::flag_words(R) * sizeof(uint32_t);
   pl.ring_off = (pl.flag_bytes + 1023) & ~static_cast<size_t>(1023);
   pl.ring_unit = static_cast<size_t>(R) * kda::pipe::SLOT;
-  pl.bytes = pl.ring_off + pl.ring_unit * kda::pipe::MAX_RING;
+  // preferred depth: as deep as kRingL2Bytes of ring allows (the ring should
+  // stay in L2 next to the streaming inputs: a deeper ring is written back to
+  // HBM), at least kMinPreferredRing slots
+  int depth = static_cast<int>(kRingL2Bytes / pl.ring_unit);
+  depth = depth < kMinPreferredRing ? kMinPreferredRing : depth;
+  depth = depth > kda::pipe::MAX_RING ? kda::pipe::MAX_RING : depth;
+  pl.bytes = pl.ring_off + pl.ring_unit * depth;
   pl.min_bytes = pl.ring_off + pl.ring_unit * 2;
   return pl;
 }

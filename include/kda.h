@@ -102,13 +102,15 @@ typedef struct kda_shape {
  * kda_chunk_fwd_workspace_size -- preferred bytes of device workspace for
  * kda_chunk_fwd with `shape` on the CURRENT device.  0 on the CUDA-core path.
  * On the tensor-core path the workspace holds a few KB of counters and an
- * operand ring of up to 16 slots of 66,560 bytes for each of R "state" CTAs
- * (R is chosen per call from the number of (sequence, head) pairs and the SM
- * count, at most one less than the SM count): at most ~160 MB on a 148-SM
- * B200, typically 20-80 MB, independent of the sequence lengths.  A smaller
- * workspace also works, down to a 2-slot ring, with a shallower and slower
- * pipeline; below that kda_chunk_fwd returns KDA_ERR_WORKSPACE.  Returns 0
- * for shapes the library rejects; kda_chunk_fwd then reports the reason.
+ * operand ring of 66,560-byte slots for each of R "state" CTAs (R is chosen
+ * per call from the number of (sequence, head) pairs and the SM count, at
+ * most one less than the SM count).  The preferred depth keeps the whole ring
+ * within about 48 MB, so that it stays in L2 next to the streaming inputs,
+ * with 4 to 16 slots per state CTA: at most ~50 MB on a 148-SM B200, and
+ * independent of the sequence lengths.  Any workspace from a 2-slot to a
+ * 16-slot ring works (deeper rings tolerate more imbalance between chains);
+ * below 2 slots kda_chunk_fwd returns KDA_ERR_WORKSPACE.  Returns 0 for shapes
+ * the library rejects; kda_chunk_fwd then reports the reason.
  */
 size_t kda_chunk_fwd_workspace_size(const kda_shape* shape);
 
