@@ -51,6 +51,8 @@ def _load():
         ]
         lib.kda_oracle_decode.restype = ctypes.c_int
         lib.kda_oracle_mutation_count.restype = ctypes.c_int
+        lib.kda_oracle_output_gate.argtypes = [ctypes.c_int64, ctypes.c_int, dp, dp, dp, ctypes.c_double, dp]
+        lib.kda_oracle_output_gate.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -114,3 +116,17 @@ def decode(q, k, v, log_alpha, beta, S, n_threads: int = 0):
     if rc != 0:
         raise ValueError("oracle rejected its arguments")
     return o, S
+
+
+def output_gate(o, g, w, eps: float):
+    """Per-head RMSNorm with weight ``w`` ([dv]) and sigmoid output gate ``g``
+    (same shape as ``o``, last axis dv), in fp64; returns an array shaped like o."""
+    o, g, w = _f64(o), _f64(g), _f64(w)
+    if o.shape != g.shape or w.shape != (o.shape[-1],):
+        raise ValueError("o and g must match; w must have dv values")
+    dv = o.shape[-1]
+    out = np.zeros_like(o)
+    rc = _load().kda_oracle_output_gate(o.size // dv, dv, _ptr(o), _ptr(g), _ptr(w), float(eps), _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments")
+    return out

@@ -240,3 +240,34 @@ int kda_oracle_decode(int N, int H, int dk, int dv, const double* q, const doubl
 }
 
 int kda_oracle_mutation_count(void) { return MUT_COUNT; }
+
+/*
+ * kda_oracle_output_gate -- the per-head output normalisation and gate that
+ * the "Kimi Linear" summary (section "Configuracao do modelo Kimi Linear")
+ * places after the operator and before the output projection: an RMSNorm per
+ * head and a data-dependent output gate.  The page gives no formula; taken
+ * here in its plainest form, per token t and head h over the dv channels:
+ *
+ *     rms     = sqrt( (1/dv) * sum_j o[j]^2 + eps )
+ *     out[j]  = o[j] / rms * w[j] * sigmoid(g[j]),   sigmoid(x) = 1 / (1 + e^-x)
+ *
+ * w (dv values) is the RMSNorm weight, shared by all heads; g is the gate's
+ * pre-activation for this token and head (the low-rank projection that
+ * produces it belongs to the model, not to the operator).
+ * o, g, out: [rows, dv] (rows = tokens x heads, one row per (token, head)).
+ */
+int kda_oracle_output_gate(int64_t rows, int dv, const double* o, const double* g, const double* w, double eps,
+                           double* out) {
+  if (rows < 0 || dv <= 0 || !o || !g || !w || !out || !(eps >= 0.0)) return -1;
+  for (int64_t r = 0; r < rows; ++r) {
+    const double* x = o + r * dv;
+    double ss = 0.0;
+    for (int j = 0; j < dv; ++j) ss += x[j] * x[j];
+    const double rms = sqrt(ss / dv + eps);
+    for (int j = 0; j < dv; ++j) {
+      const double gate = 1.0 / (1.0 + exp(-g[r * dv + j]));
+      out[r * dv + j] = x[j] / rms * w[j] * gate;
+    }
+  }
+  return 0;
+}
