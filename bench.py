@@ -266,7 +266,8 @@ def run_reference(args):
 
 PROFILE_DIR = ROOT / "profiles"
 KERNEL_SOURCES = ("gated_delta_rule_110_b200/csrc/kda_prefill.cuh", "gated_delta_rule_110_b200/csrc/kda_ptx.cuh",
-                  "gated_delta_rule_110_b200/csrc/kda_recurrent.cuh", "gated_delta_rule_110_b200/csrc/kda_api.cu")
+                  "gated_delta_rule_110_b200/csrc/kda_recurrent.cuh", "gated_delta_rule_110_b200/csrc/kda_api.cu",
+                  "gated_delta_rule_110_b200/csrc/kda_epilogue.cuh")
 
 
 def kernel_sources_hash() -> str:
@@ -306,8 +307,11 @@ def cpu_model() -> str:
     return "unknown"
 
 
-def prefill_leg(kda, gen, wname, steps, warmup, world, rank, local, stream, peaks, peak_src, counters):
-    """Times kda_chunk_fwd on one workload; returns its JSON object."""
+def prefill_leg(kda, gen, wname, steps, warmup, world, rank, local, stream, peaks, peak_src, counters,
+                gated=False):
+    """Times kda_chunk_fwd (kda_chunk_fwd_gated with ``gated``: the output
+    RMSNorm and sigmoid gate, placed by the library) on one workload; returns
+    its JSON object."""
     w = gen.workload(wname)
     x = gen.workload_inputs(w, device="cuda", seed_offset=rank)
     cu = x["cu_seqlens"]
@@ -317,28 +321,39 @@ def prefill_leg(kda, gen, wname, steps, warmup, world, rank, local, stream, peak
     ws = torch.empty(max(kda.kda_chunk_fwd_workspace_size(shape), 1), dtype=torch.uint8, device="cuda")
     o = torch.empty_like(x["v"])
     S_T = torch.empty_like(x["S0"])
+    if gated:
+        gate, nw = gen.output_gate_inputs(x["v"].shape, seed=w.seed + 100 + rank, device="cuda")
 
-    def fn():
-        kda.kda_chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["S0"], cu, o=o, S_T=S_T, workspace=ws)
+        def fn():
+            kda.kda_chunk_fwd_gated(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], gate, nw, x["S0"], cu,
+                                    eps=1e-5, o=o, S_T=S_T, workspace=ws)
+    else:
+        def fn():
+            kda.kda_chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["S0"], cu, o=o, S_T=S_T,
+                              workspace=ws)
 
-    progress(f"{wname}: timing {steps} calls")
+    label = wname + (" gated" if gated else "")
+    progress(f"{label}: timing {steps} calls")
     with ClockSampler(local) as clk:
         t = timed(fn, steps, warmup, world, stream)
     err = kda.kda_check_device_error()
     if err != 0:
-        raise RuntimeError(f"device error {err} during {wname}")
+        raise RuntimeError(f"device error {err} during {label}")
     tokens = w.B * w.T
     ms = t / steps * 1e3
     nbytes = prefill_bytes(tokens, 1, w.H, w.dk) - 2 * tokens * w.H * w.dk * w.dk * 4 + 2 * N * w.H * w.dk * w.dk * 4
+    if gated:
+        nbytes += tokens * w.H * w.dv * 2 + w.dv * 4  # the gate read, the norm weight
     flops = prefill_flops(tokens, 1, w.H, w.dk)
     gbs = nbytes / (ms / 1e3) / 1e9
     peak = float(peaks["hbm_gbs"])
-    c = counters.get(wname, {})
+    c = counters.get(wname + ("_gated" if gated else ""), {})
     traffic = c.get("dram_bytes")
-    progress(f"{wname}: {ms:.3f} ms/call, {gbs:.0f} GB/s")
+    progress(f"{label}: {ms:.3f} ms/call, {gbs:.0f} GB/s")
     out = {
         "value": tokens * world * steps / t, "unit": "tokens/s", "ms_per_step": ms, "steps": steps,
-        "config": {"workload": f"{wname} {w.B}x{w.T} tokens H{w.H} dk=dv={w.dk} C64, bf16 q/k/v/gates, fp32 state",
+        "config": {"workload": f"{wname} {w.B}x{w.T} tokens H{w.H} dk=dv={w.dk} C64, bf16 q/k/v/gates, fp32 state"
+                               + (", fused per-head RMSNorm + sigmoid output gate (bf16 gate)" if gated else ""),
                    "sequences": N, "tokens": tokens, "H": w.H,
                    "l2": f"inputs larger than L2 (no flush): {tokens * w.H * w.dk * 8 / 1e6:.0f} MB read per call"},
         "roofline": {"kernel": "kda_prefill_kernel (one cooperative launch per call)", "bound": "hbm",
@@ -350,6 +365,8 @@ def prefill_leg(kda, gen, wname, steps, warmup, world, rank, local, stream, peak
         "clocks": clk.summary(),
     }
     del x, ws, o, S_T
+    if gated:
+        del gate, nw
     torch.cuda.empty_cache()
     return out
 
@@ -409,6 +426,12 @@ def run_ours(args):
     lng = prefill_leg(kda, gen, "long", long_steps, args.warmup, world, rank, local, stream, peaks, peak_src,
                       counters)
     launches += long_steps
+    gtd = prefill_leg(kda, gen, "prefill", args.steps, args.warmup, world, rank, local, stream, peaks, peak_src,
+                      counters, gated=True)
+    launches += args.steps
+    lgt = prefill_leg(kda, gen, "long", long_steps, args.warmup, world, rank, local, stream, peaks, peak_src,
+                      counters, gated=True)
+    launches += 2 * long_steps  # the prefill kernel and the separate epilogue pass
 
     # ---------------- decode
     progress("decode: setup")
@@ -458,6 +481,8 @@ def run_ours(args):
             "clocks": pre["clocks"],
             "varlen": var,
             "long": lng,
+            "prefill_gated": gtd,
+            "long_gated": lgt,
             "decode": {"value": world * dec_steps / t_dec, "unit": "steps/s", "ms_per_step": dec_ms,
                        "steps": dec_steps,
                        "config": {"workload": "decode 256 seqs x H32 dk=dv=128, fp32 state 537 MB in place, "
@@ -485,7 +510,7 @@ def run_profile(args):
     torch.cuda.set_device(0)
     kda.load_library()
     stream = torch.cuda.current_stream()
-    w = gen.workload(args.profile)
+    w = gen.workload("prefill" if args.profile.startswith("gated") else args.profile)
     if args.profile == "decode":
         S = gen.decode_state(w.B, w.H, w.dk, w.dv, device="cuda", seed=w.seed)
         xs = gen.decode_step_inputs(w.B, w.H, w.dk, w.dv, 0, device="cuda", seed=w.seed)
@@ -501,9 +526,17 @@ def run_profile(args):
         o = torch.empty_like(x["v"])
         S_T = torch.empty_like(x["S0"])
 
+        if args.profile.startswith("gated"):
+            gate, nw = gen.output_gate_inputs(x["v"].shape, seed=w.seed + 100, device="cuda")
+            mode = "separate" if args.profile == "gated_separate" else "fused"
+
         def fn():
-            kda.kda_chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["S0"], x["cu_seqlens"], o=o,
-                              S_T=S_T, workspace=ws)
+            if args.profile.startswith("gated"):
+                kda.kda_chunk_fwd_gated(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], gate, nw, x["S0"],
+                                        x["cu_seqlens"], eps=1e-5, o=o, S_T=S_T, workspace=ws, gate_mode=mode)
+            else:
+                kda.kda_chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["S0"], x["cu_seqlens"], o=o,
+                                  S_T=S_T, workspace=ws)
     t = timed(fn, args.steps, args.warmup, 1, stream)
     err = kda.kda_check_device_error()
     print(f"{args.profile}: {t / args.steps * 1e6:.1f} us per call over {args.steps} calls, device status {err}",
@@ -524,7 +557,8 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=1000)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", choices=("prefill", "varlen", "long", "decode"), default=None,
+    ap.add_argument("--profile", choices=("prefill", "varlen", "long", "decode", "gated", "gated_separate"),
+                    default=None,
                     help="time one workload's entry point alone (for ncu); prints no JSON line")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -12,6 +12,8 @@ Entry points (same names as the C ABI):
   chunkwise-parallel prefill -> ``(o, S_T)``
 * ``kda_decode_step(q, k, v, log_alpha, beta, S)`` one recurrent token per
   (sequence, head), ``S`` updated in place -> ``o``
+* ``kda_chunk_fwd_gated(q, k, v, log_alpha, beta, out_gate, norm_weight, ...)``
+  prefill with the per-head RMSNorm and sigmoid output gate fused -> ``(o', S_T)``
 * ``kda_chunk_fwd_slots(q, k, v, log_alpha, beta, state_pool, state_slots,
   has_initial_state=None, cu_seqlens=None)`` prefill reading and writing the
   states in place in a slot-indexed pool -> ``o``
@@ -32,6 +34,9 @@ KDA_OK = 0
 KDA_F32, KDA_BF16 = 0, 1
 KDA_FLAG_VALIDATE_CU_SEQLENS = 0x1
 KDA_FLAG_PATH_RECURRENT = 0x4
+KDA_FLAG_GATE_FUSED = 0x8
+KDA_FLAG_GATE_SEPARATE = 0x10
+_GATE_MODES = {"auto": 0, "fused": KDA_FLAG_GATE_FUSED, "separate": KDA_FLAG_GATE_SEPARATE}
 
 _STATUS_NAMES = {
     0: "KDA_OK", -1: "KDA_ERR_NULL", -2: "KDA_ERR_SHAPE", -3: "KDA_ERR_DTYPE", -4: "KDA_ERR_ALIGN",
@@ -40,7 +45,8 @@ _STATUS_NAMES = {
 }
 
 EXPORTED_SYMBOLS = (
-    "kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_chunk_fwd_noalloc", "kda_chunk_fwd_slots",
+    "kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_chunk_fwd_gated", "kda_chunk_fwd_noalloc",
+    "kda_chunk_fwd_slots",
     "kda_decode_step", "kda_decode_step_slots", "kda_check_device_error", "kda_status_string",
     "kda_abi_version",
 )
@@ -84,6 +90,9 @@ def load_library(build_if_missing: bool = True):
     lib.kda_chunk_fwd_workspace_size.restype = ctypes.c_size_t
     lib.kda_chunk_fwd.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
     lib.kda_chunk_fwd.restype = ctypes.c_int
+    lib.kda_chunk_fwd_gated.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp, vp,
+                                        ctypes.c_size_t, vp]
+    lib.kda_chunk_fwd_gated.restype = ctypes.c_int
     lib.kda_chunk_fwd_noalloc.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.kda_chunk_fwd_noalloc.restype = ctypes.c_int
     lib.kda_chunk_fwd_slots.argtypes = [sp, vp, vp, vp, vp, vp, vp, ctypes.c_int32, vp, vp, vp, vp, vp,
@@ -191,6 +200,43 @@ def kda_chunk_fwd(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, *, chunk: 
         _ptr(cu_seqlens), _ptr(o), _ptr(S_T), _ptr(workspace), ws_bytes, _stream(stream))
     if rc != KDA_OK:
         raise KdaError(rc, "kda_chunk_fwd")
+    return o, S_T
+
+
+def kda_chunk_fwd_gated(q, k, v, log_alpha, beta, out_gate, norm_weight, S0=None, cu_seqlens=None, *,
+                        eps: float = 1e-5, chunk: int = 64, o=None, S_T=None, workspace=None, stream=None,
+                        validate: bool = False, output_final_state: bool = True, recurrent: bool = False,
+                        gate_mode: str = "auto", state_ctas: int = 0, grid_ctas: int = 0):
+    """Prefill followed by the per-head RMSNorm and sigmoid output gate
+    (include/kda.h, kda_chunk_fwd_gated): returns (o', S_T) with
+    o' = o / rms(o) * norm_weight * sigmoid(out_gate).  ``gate_mode``:
+    "auto" (the library decides), "fused" (in the tensor-core kernel's output
+    warps) or "separate" (a pass over o after the prefill)."""
+    import torch
+    _need_cuda(q, k, v, log_alpha, beta, out_gate, norm_weight, S0, cu_seqlens, o, S_T, workspace)
+    if out_gate.shape != v.shape or out_gate.dtype != v.dtype:
+        raise ValueError("out_gate must have the shape and dtype of v")
+    if norm_weight.dtype != torch.float32 or norm_weight.numel() != v.shape[-1]:
+        raise ValueError("norm_weight must be a float32 tensor of dv values")
+    if gate_mode not in _GATE_MODES:
+        raise ValueError(f"gate_mode must be one of {sorted(_GATE_MODES)}")
+    shape = _shape_of(q, v, log_alpha, cu_seqlens, chunk, validate, recurrent, state_ctas, grid_ctas)
+    shape.flags |= _GATE_MODES[gate_mode]
+    N = shape.B if cu_seqlens is None else shape.n_seqs
+    if o is None:
+        o = torch.empty(v.shape, dtype=v.dtype, device=v.device)
+    if S_T is None and output_final_state:
+        S_T = torch.empty((N, shape.H, shape.dk, shape.dv), dtype=torch.float32, device=q.device)
+    need = kda_chunk_fwd_workspace_size(shape)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = load_library().kda_chunk_fwd_gated(
+        ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0), _ptr(cu_seqlens),
+        _ptr(out_gate), _ptr(norm_weight), float(eps), _ptr(o), _ptr(S_T), _ptr(workspace), ws_bytes,
+        _stream(stream))
+    if rc != KDA_OK:
+        raise KdaError(rc, "kda_chunk_fwd_gated")
     return o, S_T
 
 

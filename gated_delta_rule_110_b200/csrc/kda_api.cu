@@ -33,8 +33,8 @@ inline bool dim_ok(int32_t d) { return d == 64 || d == 128; }
 inline bool use_tc(const kda_shape& s) {
   return s.io_dtype == KDA_BF16 && s.dk == 128 && s.dv == 128 && (s.flags & KDA_FLAG_PATH_RECURRENT) == 0u;
 }
-constexpr uint32_t kKnownFlags =
-    KDA_FLAG_VALIDATE_CU_SEQLENS | KDA_FLAG_PATH_RECURRENT | KDA_FLAG_STATE_CTAS(0xFF) | KDA_FLAG_GRID_CTAS(0xFF);
+constexpr uint32_t kKnownFlags = KDA_FLAG_VALIDATE_CU_SEQLENS | KDA_FLAG_PATH_RECURRENT | KDA_FLAG_GATE_FUSED |
+                                  KDA_FLAG_GATE_SEPARATE | KDA_FLAG_STATE_CTAS(0xFF) | KDA_FLAG_GRID_CTAS(0xFF);
 
 // Number of sequences N and the packed token total.
 inline void seq_counts(const kda_shape& s, const int32_t* cu, int64_t* N, int64_t* Ttot) {
@@ -54,6 +54,7 @@ kda_status check_common(const kda_shape* sp) {
   if (s.B <= 0 || s.T < 0 || s.H <= 0) return KDA_ERR_SHAPE;
   if (!dim_ok(s.dk) || !dim_ok(s.dv)) return KDA_ERR_UNSUPPORTED;
   if ((s.flags & ~kKnownFlags) != 0u) return KDA_ERR_ARGUMENT;
+  if ((s.flags & KDA_FLAG_GATE_FUSED) && (s.flags & KDA_FLAG_GATE_SEPARATE)) return KDA_ERR_ARGUMENT;
   return KDA_OK;
 }
 
@@ -126,8 +127,16 @@ int device_sm_count() {
   return n;
 }
 
+// Optional output epilogue of the tensor-core prefill (gate == nullptr: none).
+struct Epilogue {
+  const void* gate = nullptr;
+  const float* norm_w = nullptr;
+  float eps = 0.f;
+};
+
 struct PrefillPlan {
   int R = 0;             // state CTAs
+  bool fuse_gate = false;  // output epilogue in the state CTAs (they have time to spare)
   int grid = 0;          // all CTAs (one per SM)
   size_t flag_bytes = 0; // zeroed before each launch
   size_t ring_off = 0;
@@ -149,6 +158,10 @@ struct PrefillPlan {
 // kTransformCost times as long per chunk as a state CTA spends on one chunk
 // of its chain.  R minimises the larger of the two times.
 constexpr double kTransformCost = 2.0;
+// A state CTA with the output epilogue fused spends about kFusedGateCost
+// times as long per chunk; the epilogue is fused where that still does not
+// make the state CTAs the bound, else it runs as a separate pass over o.
+constexpr double kFusedGateCost = 1.5;
 constexpr size_t kRingL2Bytes = 48u << 20;
 constexpr int kMinPreferredRing = 4;
 
@@ -177,6 +190,11 @@ PrefillPlan plan_prefill(const kda_shape& s, int64_t N, int nsm) {
   }
   pl.R = R;
   pl.grid = grid;
+  {
+    const double t_state = static_cast<double>((chains + R - 1) / R);
+    const double t_tf = static_cast<double>(chains) * kTransformCost / (grid - R);
+    pl.fuse_gate = t_state * kFusedGateCost <= t_tf;
+  }
   pl.flag_bytes = kda::pipe::flag_words(R) * sizeof(uint32_t);
   pl.ring_off = (pl.flag_bytes + 1023) & ~static_cast<size_t>(1023);
   pl.ring_unit = static_cast<size_t>(R) * kda::pipe::SLOT;
@@ -191,12 +209,19 @@ PrefillPlan plan_prefill(const kda_shape& s, int64_t N, int nsm) {
   return pl;
 }
 
+// With an epilogue, *fused says whether the kernel applied it (else the caller
+// runs the separate pass).
 template <typename TG>
 kda_status launch_prefill(const kda_shape& s, int64_t N, int64_t Ttot, const void* q, const void* k, const void* v,
-                          const void* la, const void* beta, const kda::StateIO& io, const int32_t* cu, void* o,
-                          void* ws, size_t ws_bytes, cudaStream_t st) {
+                          const void* la, const void* beta, const kda::StateIO& io, const Epilogue& ep_req,
+                          const int32_t* cu, void* o,
+                          void* ws, size_t ws_bytes, cudaStream_t st, bool* fused) {
   namespace P = kda::pipe;
   const PrefillPlan pl = plan_prefill(s, N, device_sm_count());
+  const bool fuse = ep_req.gate != nullptr && ((s.flags & KDA_FLAG_GATE_FUSED) != 0u ||
+                                               ((s.flags & KDA_FLAG_GATE_SEPARATE) == 0u && pl.fuse_gate));
+  const Epilogue ep = fuse ? ep_req : Epilogue{};
+  *fused = fuse;
   if (pl.R <= 0) return KDA_ERR_CUDA;
   const int nring = pl.nring(ws_bytes);
   if (!ws || nring < 2) return KDA_ERR_WORKSPACE;
@@ -226,9 +251,12 @@ kda_status launch_prefill(const kda_shape& s, int64_t N, int64_t Ttot, const voi
   prm.beta = beta;
   prm.st = io;
   prm.o = static_cast<__nv_bfloat16*>(o);
+  prm.gate = static_cast<const __nv_bfloat16*>(ep.gate);
+  prm.norm_w = ep.norm_w;
+  prm.eps = ep.eps;
   prm.flags = static_cast<uint32_t*>(ws);
   prm.ring = static_cast<uint8_t*>(ws) + pl.ring_off;
-  auto* kern = P::kda_prefill_kernel<TG>;
+  auto* kern = ep.gate ? P::kda_prefill_kernel<TG, true> : P::kda_prefill_kernel<TG, false>;
   const uint32_t smem = P::ST_BYTES > P::TfLayout<TG>::BYTES ? P::ST_BYTES : P::TfLayout<TG>::BYTES;
   if (!ensure_smem(kern, smem)) return KDA_ERR_CUDA;
   if (cudaMemsetAsync(ws, 0, pl.flag_bytes, st) != cudaSuccess) return KDA_ERR_CUDA;
@@ -247,6 +275,23 @@ kda_status launch_prefill(const kda_shape& s, int64_t N, int64_t Ttot, const voi
     return KDA_ERR_CUDA;
   }
   return KDA_OK;
+}
+
+// The output epilogue as its own pass over o (kda_epilogue.cuh).
+template <typename TO>
+kda_status launch_output_gate(TO* o, const void* gate, const float* w, float eps, int64_t rows, int dv,
+                              cudaStream_t st) {
+  namespace E = kda::epi;
+  const int rows_per_block = E::kThreads / (dv / 8);
+  const int64_t want = (rows + 2 * rows_per_block - 1) / (2 * rows_per_block);
+  const int64_t cap = static_cast<int64_t>(device_sm_count()) * 8;
+  const unsigned blocks = static_cast<unsigned>(want < cap ? (want > 0 ? want : 1) : (cap > 0 ? cap : 1));
+  const TO* g = static_cast<const TO*>(gate);
+  if (dv == 128)
+    E::kda_output_gate_kernel<TO, 128><<<blocks, E::kThreads, 0, st>>>(o, g, w, eps, rows);
+  else
+    E::kda_output_gate_kernel<TO, 64><<<blocks, E::kThreads, 0, st>>>(o, g, w, eps, rows);
+  return launch_status();
 }
 
 kda_status validate_cu_host(const int32_t* cu, int64_t N, int64_t Ttot, cudaStream_t st) {
@@ -290,7 +335,8 @@ size_t kda_chunk_fwd_min_workspace(const kda_shape* sp) {
 // Shared body of kda_chunk_fwd and kda_chunk_fwd_slots; `io` says where the
 // states live (dense rows or pool slots).
 kda_status chunk_fwd(const kda_shape* sp, const void* q, const void* k, const void* v, const void* log_alpha,
-                     const void* beta, const kda::StateIO& io, const int32_t* cu_seqlens, void* o, void* workspace,
+                     const void* beta, const kda::StateIO& io, const Epilogue& ep, const int32_t* cu_seqlens,
+                     void* o, void* workspace,
                      size_t workspace_bytes, void* stream) {
   kda_status e = check_common(sp);
   if (e != KDA_OK) return e;
@@ -311,24 +357,34 @@ kda_status chunk_fwd(const kda_shape* sp, const void* q, const void* k, const vo
   }
   if (N == 0) return KDA_OK;
 
+  if (ep.gate && Ttot > 0 && (!aligned16(o) || !aligned16(ep.gate))) return KDA_ERR_ALIGN;
+  bool fused = false;
   if (use_tc(s) && Ttot > 0) {
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(log_alpha) || !aligned16(o))
       return KDA_ERR_ALIGN;
     if (s.gate_dtype == KDA_BF16)
-      return launch_prefill<__nv_bfloat16>(s, N, Ttot, q, k, v, log_alpha, beta, io, cu_seqlens, o, workspace,
-                                           workspace_bytes, st);
-    return launch_prefill<float>(s, N, Ttot, q, k, v, log_alpha, beta, io, cu_seqlens, o, workspace,
-                                 workspace_bytes, st);
-  }
-  if (s.io_dtype == KDA_F32) {
+      e = launch_prefill<__nv_bfloat16>(s, N, Ttot, q, k, v, log_alpha, beta, io, ep, cu_seqlens, o, workspace,
+                                        workspace_bytes, st, &fused);
+    else
+      e = launch_prefill<float>(s, N, Ttot, q, k, v, log_alpha, beta, io, ep, cu_seqlens, o, workspace,
+                                workspace_bytes, st, &fused);
+  } else if (s.io_dtype == KDA_F32) {
     if (s.gate_dtype == KDA_F32)
-      return dispatch_recurrent_fwd<float, float>(s, N, q, k, v, log_alpha, beta, io, cu_seqlens, o, st);
-    return dispatch_recurrent_fwd<float, __nv_bfloat16>(s, N, q, k, v, log_alpha, beta, io, cu_seqlens, o, st);
+      e = dispatch_recurrent_fwd<float, float>(s, N, q, k, v, log_alpha, beta, io, cu_seqlens, o, st);
+    else
+      e = dispatch_recurrent_fwd<float, __nv_bfloat16>(s, N, q, k, v, log_alpha, beta, io, cu_seqlens, o, st);
+  } else if (s.gate_dtype == KDA_F32) {
+    e = dispatch_recurrent_fwd<__nv_bfloat16, float>(s, N, q, k, v, log_alpha, beta, io, cu_seqlens, o, st);
+  } else {
+    e = dispatch_recurrent_fwd<__nv_bfloat16, __nv_bfloat16>(s, N, q, k, v, log_alpha, beta, io, cu_seqlens, o,
+                                                             st);
   }
-  if (s.gate_dtype == KDA_F32)
-    return dispatch_recurrent_fwd<__nv_bfloat16, float>(s, N, q, k, v, log_alpha, beta, io, cu_seqlens, o, st);
-  return dispatch_recurrent_fwd<__nv_bfloat16, __nv_bfloat16>(s, N, q, k, v, log_alpha, beta, io, cu_seqlens, o,
-                                                              st);
+  if (e != KDA_OK || !ep.gate || fused || Ttot == 0) return e;
+  const int64_t rows = Ttot * s.H;
+  if (s.io_dtype == KDA_F32)
+    return launch_output_gate<float>(static_cast<float*>(o), ep.gate, ep.norm_w, ep.eps, rows, s.dv, st);
+  return launch_output_gate<__nv_bfloat16>(static_cast<__nv_bfloat16*>(o), ep.gate, ep.norm_w, ep.eps, rows, s.dv,
+                                           st);
 }
 
 // Shared body of kda_decode_step and kda_decode_step_slots.
@@ -363,7 +419,8 @@ kda_status kda_chunk_fwd(const kda_shape* sp, const void* q, const void* k, cons
   kda::StateIO io;
   io.S0 = S0;
   io.S_T = S_T;
-  return chunk_fwd(sp, q, k, v, log_alpha, beta, io, cu_seqlens, o, workspace, workspace_bytes, stream);
+  return chunk_fwd(sp, q, k, v, log_alpha, beta, io, Epilogue{}, cu_seqlens, o, workspace, workspace_bytes,
+                   stream);
 }
 
 kda_status kda_chunk_fwd_slots(const kda_shape* sp, const void* q, const void* k, const void* v,
@@ -380,7 +437,26 @@ kda_status kda_chunk_fwd_slots(const kda_shape* sp, const void* q, const void* k
   io.slots = state_slots;
   io.has_init = has_initial_state;
   io.num_slots = num_slots;
-  return chunk_fwd(sp, q, k, v, log_alpha, beta, io, cu_seqlens, o, workspace, workspace_bytes, stream);
+  return chunk_fwd(sp, q, k, v, log_alpha, beta, io, Epilogue{}, cu_seqlens, o, workspace, workspace_bytes,
+                   stream);
+}
+
+kda_status kda_chunk_fwd_gated(const kda_shape* sp, const void* q, const void* k, const void* v,
+                               const void* log_alpha, const void* beta, const float* S0, const int32_t* cu_seqlens,
+                               const void* out_gate, const float* norm_weight, float eps, void* o, float* S_T,
+                               void* workspace, size_t workspace_bytes, void* stream) {
+  if (!sp) return KDA_ERR_NULL;
+  if (!out_gate || !norm_weight) return KDA_ERR_NULL;
+  if (!(eps >= 0.f) || !(eps < 3.0e38f)) return KDA_ERR_ARGUMENT;
+  if (!aligned16(out_gate) || !aligned16(norm_weight)) return KDA_ERR_ALIGN;
+  kda::StateIO io;
+  io.S0 = S0;
+  io.S_T = S_T;
+  Epilogue ep;
+  ep.gate = out_gate;
+  ep.norm_w = norm_weight;
+  ep.eps = eps;
+  return chunk_fwd(sp, q, k, v, log_alpha, beta, io, ep, cu_seqlens, o, workspace, workspace_bytes, stream);
 }
 
 kda_status kda_decode_step(const kda_shape* sp, const void* q, const void* k, const void* v, const void* log_alpha,

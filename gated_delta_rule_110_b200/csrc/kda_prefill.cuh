@@ -43,6 +43,7 @@
 // that every CTA polls.
 #pragma once
 
+#include "kda_epilogue.cuh"
 #include "kda_ptx.cuh"
 #include "kda_state_io.cuh"
 
@@ -151,6 +152,11 @@ struct Params {
   const void* beta;
   StateIO st;       // initial / final states (dense rows or pool slots)
   __nv_bfloat16* o;
+  // optional output epilogue (gate == nullptr: o is written as computed):
+  // o <- o / rms(o) * norm_w * sigmoid(gate), rms over the head's dv values
+  const __nv_bfloat16* gate;  // [B, T, H, dv], like o
+  const float* norm_w;        // [dv]
+  float eps;
   int nring;        // ring slots per state CTA, 2..MAX_RING
   uint8_t* ring;    // R * nring slots
   uint32_t* flags;  // flag_words(R), zero on entry
@@ -1096,6 +1102,13 @@ __device__ __forceinline__ void state_mma_loop(uint32_t sbase, uint32_t tmem, co
 // chunk (TMEM lanes 64 + 32 u + lane), 128 values each.  Each warp stages its
 // 32 x 128 block as bf16 in shared memory and stores it with two tensor
 // stores when all its rows belong to the sequence, else row by row.
+//
+// GATED: the output epilogue of the Kimi Linear layer, o <- o / rms(o) *
+// norm_w * sigmoid(gate) per (token, head) row.  A lane reads its row from
+// TMEM twice (the mean square first; holding all 128 values measured
+// slower), and fetches its row of the gate into its own row of the staging
+// block (where its outputs go) while the products are still being formed.
+template <bool GATED>
 __device__ __forceinline__ void state_output_loop(uint8_t* smem, uint32_t tmem, const Maps& maps, const Params& p,
                                                   uint64_t* bars, volatile int* abort_flag) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -1112,26 +1125,88 @@ __device__ __forceinline__ void state_output_loop(uint8_t* smem, uint32_t tmem, 
       const int b = pos & 1;
       const int64_t t0 = w.sb + static_cast<int64_t>(j) * C;
       const int L = static_cast<int>(w.se - t0 < C ? w.se - t0 : C);
-      if (!mbar_wait_warp(&bars[BS_O_FULL + b], (pos >> 1) & 1, abort_flag)) { ok = false; break; }
-      tc_fence_after();
-      // the previous tensor store out of the staging block must have read it
-      if (lane == 0) bulk_wait_read<0>();
-      __syncwarp();
-#pragma unroll 1
-      for (int cb = 0; cb < 4; ++cb) {
-        float x[32];
-        tmem_ld32(tmem + lane_off + TS_O + 128 * b + 32 * cb, x);
-        tmem_wait_ld();
+      if constexpr (GATED) {
+        // the previous tensor store out of the staging block must have read it
+        if (lane == 0) bulk_wait_read<0>();
+        __syncwarp();
+        if (r < L) {
+          const __nv_bfloat16* grow = p.gate + ((t0 + r) * p.H + h) * D;
 #pragma unroll
-        for (int j4 = 0; j4 < 4; ++j4) {
-          const int vv = 32 * cb + 8 * j4;
-          sts128(st + (vv >> 6) * 4096 + sw128(lane, (vv & 63) >> 3),
-                 make_uint4(pack_bf16(x[8 * j4], x[8 * j4 + 1]), pack_bf16(x[8 * j4 + 2], x[8 * j4 + 3]),
-                            pack_bf16(x[8 * j4 + 4], x[8 * j4 + 5]), pack_bf16(x[8 * j4 + 6], x[8 * j4 + 7])));
+          for (int c16 = 0; c16 < 16; ++c16)
+            cp_async16(st + (c16 >> 3) * 4096 + sw128(lane, c16 & 7), grow + 8 * c16);
         }
+        cp_async_commit();
       }
-      tc_fence_before();
-      mbar_arrive(&bars[BS_O_FREE + b]);
+      if (!mbar_wait_warp(&bars[BS_O_FULL + b], (pos >> 1) & 1, abort_flag)) {
+        if constexpr (GATED) cp_async_wait_all();
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      if constexpr (GATED) {
+        // the row's mean square (one pass over TMEM), then the products again
+        float ss0 = 0.f, ss1 = 0.f;
+#pragma unroll 1
+        for (int cb = 0; cb < 4; ++cb) {
+          float x[32];
+          tmem_ld32(tmem + lane_off + TS_O + 128 * b + 32 * cb, x);
+          tmem_wait_ld();
+#pragma unroll
+          for (int u = 0; u < 32; u += 2) {
+            ss0 = fmaf(x[u], x[u], ss0);
+            ss1 = fmaf(x[u + 1], x[u + 1], ss1);
+          }
+        }
+        const float rinv = rsqrtf((ss0 + ss1) * (1.f / D) + p.eps);
+        cp_async_wait_all();
+#pragma unroll 1
+        for (int cb = 0; cb < 4; ++cb) {
+          float x[32];
+          tmem_ld32(tmem + lane_off + TS_O + 128 * b + 32 * cb, x);
+          tmem_wait_ld();
+          // o / rms * w * sigmoid(g), the gate read from where the result goes
+          // (rows past the sequence end hold stale values and are not written)
+#pragma unroll
+          for (int j4 = 0; j4 < 4; ++j4) {
+            const int c0 = 32 * cb + 8 * j4;
+            uint8_t* at = st + (c0 >> 6) * 4096 + sw128(lane, (c0 & 63) >> 3);
+            const uint4 gw = lds128(at);
+            const uint32_t g4[4] = {gw.x, gw.y, gw.z, gw.w};
+            const float4 wa = __ldg(reinterpret_cast<const float4*>(p.norm_w + c0));
+            const float4 wb = __ldg(reinterpret_cast<const float4*>(p.norm_w + c0 + 4));
+            const float w8[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+            uint32_t pk[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const float2 gv = bf2f(g4[u]);
+              pk[u] = pack_bf16(x[8 * j4 + 2 * u] * rinv * w8[2 * u] * epi::sigmoid_tanh(gv.x),
+                                x[8 * j4 + 2 * u + 1] * rinv * w8[2 * u + 1] * epi::sigmoid_tanh(gv.y));
+            }
+            sts128(at, make_uint4(pk[0], pk[1], pk[2], pk[3]));
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&bars[BS_O_FREE + b]);
+      } else {
+        // the previous tensor store out of the staging block must have read it
+        if (lane == 0) bulk_wait_read<0>();
+        __syncwarp();
+#pragma unroll 1
+        for (int cb = 0; cb < 4; ++cb) {
+          float x[32];
+          tmem_ld32(tmem + lane_off + TS_O + 128 * b + 32 * cb, x);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j4 = 0; j4 < 4; ++j4) {
+            const int vv = 32 * cb + 8 * j4;
+            sts128(st + (vv >> 6) * 4096 + sw128(lane, (vv & 63) >> 3),
+                   make_uint4(pack_bf16(x[8 * j4], x[8 * j4 + 1]), pack_bf16(x[8 * j4 + 2], x[8 * j4 + 3]),
+                              pack_bf16(x[8 * j4 + 4], x[8 * j4 + 5]), pack_bf16(x[8 * j4 + 6], x[8 * j4 + 7])));
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&bars[BS_O_FREE + b]);
+      }
       if (32 * sub + 32 <= L) {
         fence_proxy_async_smem();
         __syncwarp();
@@ -1258,7 +1333,7 @@ __device__ __forceinline__ void state_warps_loop(uint8_t* smem, uint32_t tmem, c
 // ===========================================================================
 // the kernel
 // ===========================================================================
-template <typename TG>
+template <typename TG, bool GATED>
 __global__ void __launch_bounds__(NTHREADS, 1)
     kda_prefill_kernel(const __grid_constant__ Maps maps, const Params p) {
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -1344,7 +1419,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     } else if (warp == 9) {
       if (lane == 0) state_mma_loop(sbase, tmem, p, bars, abort_flag);
     } else {
-      state_output_loop(smem, tmem, maps, p, bars, abort_flag);
+      state_output_loop<GATED>(smem, tmem, maps, p, bars, abort_flag);
     }
   } else {
     const int g = (warp < 8) ? (warp >> 2) : ((warp - 8) & 1);

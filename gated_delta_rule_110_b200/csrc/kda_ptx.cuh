@@ -364,6 +364,15 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&r)[16]) {
       : "r"(taddr));
 }
 
+// Per-thread 16-byte asynchronous copy global -> shared (cached in L2 only);
+// both addresses 16-byte aligned.  Completion: cp_async_commit, then
+// cp_async_wait_all by the same thread.
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
 // 2^x on the MUFU unit (approximate, flush-to-zero).
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;

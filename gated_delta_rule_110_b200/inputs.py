@@ -141,6 +141,17 @@ def make_inputs(B: int, T: int, H: int, dk: int, dv: int, *, dtype=torch.bfloat1
     return dict(q=q, k=k, v=v, log_alpha=la, beta=beta, S0=S0, cu_seqlens=cu)
 
 
+def output_gate_inputs(v_shape, *, dtype=torch.bfloat16, scale: float = 2.0, seed: int = 0,
+                       device="cpu"):
+    """Inputs of the fused output epilogue: the gate's pre-activation g (shaped
+    like v, normal with standard deviation ``scale``, in ``dtype``) and the
+    per-channel RMSNorm weight w (fp32, uniform in [0.5, 1.5], dv values)."""
+    g = torch.Generator(device=device).manual_seed(seed)
+    gate = (scale * _normal(tuple(v_shape), g, device)).to(dtype)
+    w = 0.5 + torch.rand((v_shape[-1],), generator=g, device=device)
+    return gate, w
+
+
 def workload_inputs(w: Workload, device="cpu", seed_offset: int = 0) -> dict:
     """Inputs for a named workload (``workload(name)``)."""
     return make_inputs(w.B, w.T, w.H, w.dk, w.dv, dtype=w.dtype, gate=w.gate, s0=w.s0,

@@ -52,7 +52,7 @@
 extern "C" {
 #endif
 
-#define KDA_ABI_VERSION 3
+#define KDA_ABI_VERSION 4
 
 typedef enum {
   KDA_OK = 0,
@@ -90,6 +90,12 @@ typedef struct kda_shape {
  * the tensor-core path applies; fp32 io and dk or dv = 64 always take it.  A
  * reference path for validation, not a fast one. */
 #define KDA_FLAG_PATH_RECURRENT 0x4u
+/* Where kda_chunk_fwd_gated applies its output epilogue on the tensor-core
+ * path (neither: the library decides from the CTA split; both: invalid).
+ * FUSED: in the prefill kernel's output warps; SEPARATE: in a pass over o
+ * after the prefill.  Other flags are ignored by the other entry points. */
+#define KDA_FLAG_GATE_FUSED 0x8u
+#define KDA_FLAG_GATE_SEPARATE 0x10u
 /* Tuning of the tensor-core path (0 = automatic): KDA_FLAG_STATE_CTAS(n)
  * fixes the number of state CTAs (each walks whole (sequence, head) chains),
  * KDA_FLAG_GRID_CTAS(n) caps the number of CTAs of the launch (at most one per
@@ -146,6 +152,35 @@ kda_status kda_chunk_fwd(const kda_shape* shape, const void* q, const void* k, c
                          const void* log_alpha, const void* beta, const float* S0,
                          const int32_t* cu_seqlens, void* o, float* S_T, void* workspace,
                          size_t workspace_bytes, void* stream);
+
+/*
+ * kda_chunk_fwd_gated -- kda_chunk_fwd followed by the per-head output
+ * normalisation and gate that the "Kimi Linear" summary
+ * (section "Configuracao do modelo Kimi Linear") applies after the operator
+ * and before the output projection: an RMSNorm per head and a data-dependent
+ * output gate.  The page gives no formula; this call computes, for every
+ * token t and head h, over the dv values of o_t:
+ *
+ *     o'_t = o_t / sqrt(mean_j(o_t[j]^2) + eps) * norm_weight * sigmoid(g_t)
+ *
+ * and writes o' (io_dtype) to `o` in place of o_t; S_T is unchanged.
+ *
+ *   out_gate     g, [B, T, H, dv] in io_dtype (the gate's pre-activation, from
+ *                the model's low-rank projection); 16-byte aligned.
+ *   norm_weight  [dv] fp32, shared by all heads; 16-byte aligned.
+ *   eps          >= 0, added to the mean square.
+ * Everything else as kda_chunk_fwd, on every path.  The tensor-core prefill
+ * applies the epilogue in its output warps where its state CTAs have time
+ * to spare (short, many sequences), else, and on the CUDA-core paths, a
+ * second kernel on `stream` applies it to o in place (reads o and g, writes
+ * o).  KDA_FLAG_GATE_FUSED / KDA_FLAG_GATE_SEPARATE force either.  The
+ * sigmoid is computed as (1 + tanh(g/2)) / 2 with the hardware tanh
+ * approximation: within about 2.5e-4 absolute.
+ */
+kda_status kda_chunk_fwd_gated(const kda_shape* shape, const void* q, const void* k, const void* v,
+                               const void* log_alpha, const void* beta, const float* S0, const int32_t* cu_seqlens,
+                               const void* out_gate, const float* norm_weight, float eps, void* o, float* S_T,
+                               void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * kda_chunk_fwd_noalloc -- kda_chunk_fwd for callers that cannot allocate.

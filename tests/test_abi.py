@@ -30,7 +30,7 @@ def test_library_loads_and_exports_every_declared_symbol():
     lib = kda.load_library()
     for name in declared_functions():
         assert hasattr(lib, name), name
-    assert kda.kda_abi_version() == 3
+    assert kda.kda_abi_version() == 4
 
 
 def test_status_strings():
@@ -157,6 +157,30 @@ def test_slot_decode_host_validation():
     assert call(s1, f, 0, f) == -2
     assert call(kda.make_shape(4, 2, 2, 128, 128), f, 4, f) == -2
     assert call(s1, f, 4, ctypes.c_void_p(FAKE + 2)) == -4
+
+
+def call_fwd_gated(shape, gate=FAKE, weight=FAKE, eps=1e-5):
+    lib = kda.load_library()
+    vp = lambda x: None if x is None else ctypes.c_void_p(x)
+    f = vp(FAKE)
+    return lib.kda_chunk_fwd_gated(ctypes.byref(shape), f, f, f, f, f, None, None, vp(gate), vp(weight),
+                                   ctypes.c_float(eps), f, None, None, 0, None)
+
+
+def test_gated_prefill_host_validation():
+    assert call_fwd_gated(tc_shape(), gate=None) == -1
+    assert call_fwd_gated(tc_shape(), weight=None) == -1
+    assert call_fwd_gated(tc_shape(), eps=-1.0) == -10
+    assert call_fwd_gated(tc_shape(), eps=float("nan")) == -10
+    assert call_fwd_gated(tc_shape(), eps=float("inf")) == -10
+    assert call_fwd_gated(tc_shape(), gate=FAKE + 2) == -4
+    assert call_fwd_gated(tc_shape(), weight=FAKE + 4) == -4
+    assert call_fwd_gated(tc_shape(flags=kda.KDA_FLAG_GATE_FUSED | kda.KDA_FLAG_GATE_SEPARATE)) == -10
+    # every path takes the epilogue: these get as far as the launch (which
+    # fails on a machine without a GPU)
+    for shape in (tc_shape(io_dtype=0), tc_shape(dk=64, dv=64), tc_shape(flags=kda.KDA_FLAG_PATH_RECURRENT),
+                  tc_shape(B=2, T=200), tc_shape(flags=kda.KDA_FLAG_GATE_SEPARATE)):
+        assert call_fwd_gated(shape) in (-6, -7)
 
 
 def test_python_binding_refuses_cpu_tensors():
