@@ -228,7 +228,7 @@ kda_status launch_prefill(const kda_shape& s, int64_t N, int64_t Ttot, const voi
   // the work-item counter is 32-bit: R * (chunks of the longest stream) must fit
   if (static_cast<double>(pl.R) * (static_cast<double>(Ttot) / P::C + static_cast<double>(N)) > 2.0e9)
     return KDA_ERR_SHAPE;
-  P::Maps maps;
+  P::Maps maps = {};
   const uint64_t cols = static_cast<uint64_t>(s.H) * P::D;
   const uint64_t rows = static_cast<uint64_t>(Ttot);
   const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
@@ -236,6 +236,7 @@ kda_status launch_prefill(const kda_shape& s, int64_t N, int64_t Ttot, const voi
             kda::make_tma_2d(&maps.k, k, bf, 2, cols, rows, cols * 2, 64, 64) &&
             kda::make_tma_2d(&maps.v, v, bf, 2, cols, rows, cols * 2, 64, 64) &&
             kda::make_tma_2d(&maps.o, o, bf, 2, cols, rows, cols * 2, 64, 32);
+  if (ep.gate) ok = ok && kda::make_tma_2d(&maps.g, ep.gate, bf, 2, cols, rows, cols * 2, 64, 32);
   if (sizeof(TG) == 2)
     ok = ok && kda::make_tma_2d(&maps.la, la, bf, 2, cols, rows, cols * 2, 64, 64);
   else

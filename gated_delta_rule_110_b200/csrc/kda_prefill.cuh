@@ -95,7 +95,9 @@ constexpr uint32_t ST_S = ST_B + 2 * SLOT_B;       // S'^T [v][c] bf16, two 64-c
 constexpr uint32_t ST_U = ST_S + 32768;           // U^T [v][r] bf16
 constexpr uint32_t ST_OX = ST_U + 16384;          // O staging of the two output warps, 2 x [32 rows][128 v] bf16
 constexpr uint32_t ST_BAR = ST_OX + 16384;
-constexpr uint32_t ST_BYTES = ST_BAR + 256;
+constexpr uint32_t ST_W = ST_BAR + 256;           // output epilogue: norm weight fp32[128]
+constexpr uint32_t ST_BYTES = ST_W + 512;
+static_assert(ST_BYTES <= 227u * 1024u, "state CTA shared memory");
 // TMEM columns
 constexpr uint32_t TS_U = 0;     // U^T fp32                       64
 constexpr uint32_t TS_DS = 128;  // dS^T fp32                     128
@@ -140,7 +142,7 @@ enum {
 // state mbarriers
 enum {
   BS_A_FULL = 0, BS_A_FREE = 2, BS_B_FULL = 4, BS_B_FREE = 6, BS_S_READY = 8, BS_U_FULL, BS_U_READY, BS_DS_FULL, BS_SP_FREE, BS_O_FULL,
-  BS_O_FREE = BS_O_FULL + 2, BS_FIN = BS_O_FREE + 2, BS_COUNT
+  BS_O_FREE = BS_O_FULL + 2, BS_FIN = BS_O_FREE + 2, BS_G_FULL = BS_FIN + 1, BS_COUNT = BS_G_FULL + 2
 };
 
 struct Params {
@@ -165,6 +167,7 @@ struct Params {
 struct Maps {
   CUtensorMap q, k, v, la;
   CUtensorMap o;  // output, box of 64 values x 32 rows
+  CUtensorMap g;  // output gate (fused epilogue only), like o
 };
 
 // --------------------------------------------------------------------------- helpers
@@ -1098,16 +1101,25 @@ __device__ __forceinline__ void state_mma_loop(uint32_t sbase, uint32_t tmem, co
   }
 }
 
+// Waits, with a bound and regardless of the abort flag, for a tile load in
+// flight into shared memory to land (a CTA must not end with one pending).
+__device__ __forceinline__ void drain_tile(uint64_t* bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity) && clock64() - t0 < kWaitCycles) {
+  }
+}
+
 // Warps 10 and 11 write O: warp 10 + u holds output rows 32 u + lane of a
 // chunk (TMEM lanes 64 + 32 u + lane), 128 values each.  Each warp stages its
 // 32 x 128 block as bf16 in shared memory and stores it with two tensor
 // stores when all its rows belong to the sequence, else row by row.
 //
 // GATED: the output epilogue of the Kimi Linear layer, o <- o / rms(o) *
-// norm_w * sigmoid(gate) per (token, head) row.  A lane reads its row from
-// TMEM twice (the mean square first; holding all 128 values measured
-// slower), and fetches its row of the gate into its own row of the staging
-// block (where its outputs go) while the products are still being formed.
+// norm_w * sigmoid(gate) per (token, head) row.  The warp's 32 x 128 gate
+// tile comes by TMA into the staging block (where the outputs go, in the
+// same swizzled layout) while the products are still being formed; the
+// weight sits in shared memory.  A lane reads its row from TMEM twice (the
+// mean square first; holding all 128 values measured slower).
 template <bool GATED>
 __device__ __forceinline__ void state_output_loop(uint8_t* smem, uint32_t tmem, const Maps& maps, const Params& p,
                                                   uint64_t* bars, volatile int* abort_flag) {
@@ -1126,19 +1138,21 @@ __device__ __forceinline__ void state_output_loop(uint8_t* smem, uint32_t tmem, 
       const int64_t t0 = w.sb + static_cast<int64_t>(j) * C;
       const int L = static_cast<int>(w.se - t0 < C ? w.se - t0 : C);
       if constexpr (GATED) {
-        // the previous tensor store out of the staging block must have read it
-        if (lane == 0) bulk_wait_read<0>();
+        // the previous tensor store out of the staging block must have read
+        // it; then the chunk's 32 x 128 gate tile comes into it by TMA (rows
+        // past the sequence end bring other rows or zeros: never stored)
+        fence_proxy_async_smem();  // the last row-by-row pass read the block
         __syncwarp();
-        if (r < L) {
-          const __nv_bfloat16* grow = p.gate + ((t0 + r) * p.H + h) * D;
-#pragma unroll
-          for (int c16 = 0; c16 < 16; ++c16)
-            cp_async16(st + (c16 >> 3) * 4096 + sw128(lane, c16 & 7), grow + 8 * c16);
+        if (lane == 0) {
+          bulk_wait_read<0>();
+          mbar_arrive_expect_tx(&bars[BS_G_FULL + sub], 8192);
+          tma_load_2d(st, &maps.g, h * D, static_cast<int>(t0) + 32 * sub, &bars[BS_G_FULL + sub]);
+          tma_load_2d(st + 4096, &maps.g, h * D + 64, static_cast<int>(t0) + 32 * sub, &bars[BS_G_FULL + sub]);
         }
-        cp_async_commit();
+        __syncwarp();
       }
       if (!mbar_wait_warp(&bars[BS_O_FULL + b], (pos >> 1) & 1, abort_flag)) {
-        if constexpr (GATED) cp_async_wait_all();
+        if constexpr (GATED) drain_tile(&bars[BS_G_FULL + sub], pos & 1);
         ok = false;
         break;
       }
@@ -1147,34 +1161,46 @@ __device__ __forceinline__ void state_output_loop(uint8_t* smem, uint32_t tmem, 
         // the row's mean square (one pass over TMEM), then the products again
         float ss0 = 0.f, ss1 = 0.f;
 #pragma unroll 1
-        for (int cb = 0; cb < 4; ++cb) {
-          float x[32];
-          tmem_ld32(tmem + lane_off + TS_O + 128 * b + 32 * cb, x);
+        for (int cb = 0; cb < 4; cb += 2) {
+          float x[64];
+          tmem_ld32(tmem + lane_off + TS_O + 128 * b + 32 * cb, *reinterpret_cast<float (*)[32]>(x));
+          tmem_ld32(tmem + lane_off + TS_O + 128 * b + 32 * cb + 32, *reinterpret_cast<float (*)[32]>(x + 32));
           tmem_wait_ld();
 #pragma unroll
-          for (int u = 0; u < 32; u += 2) {
+          for (int u = 0; u < 64; u += 2) {
             ss0 = fmaf(x[u], x[u], ss0);
             ss1 = fmaf(x[u + 1], x[u + 1], ss1);
           }
         }
         const float rinv = rsqrtf((ss0 + ss1) * (1.f / D) + p.eps);
-        cp_async_wait_all();
+        if (!mbar_wait_warp(&bars[BS_G_FULL + sub], pos & 1, abort_flag)) {
+          drain_tile(&bars[BS_G_FULL + sub], pos & 1);
+          ok = false;
+          break;
+        }
+        const float* wsm = reinterpret_cast<const float*>(smem + ST_W);
 #pragma unroll 1
         for (int cb = 0; cb < 4; ++cb) {
           float x[32];
           tmem_ld32(tmem + lane_off + TS_O + 128 * b + 32 * cb, x);
-          tmem_wait_ld();
-          // o / rms * w * sigmoid(g), the gate read from where the result goes
-          // (rows past the sequence end hold stale values and are not written)
+          // the gate and weight of these 32 values, read while TMEM is
+          uint4 gq[4];
+          float4 wq[8];
 #pragma unroll
           for (int j4 = 0; j4 < 4; ++j4) {
             const int c0 = 32 * cb + 8 * j4;
-            uint8_t* at = st + (c0 >> 6) * 4096 + sw128(lane, (c0 & 63) >> 3);
-            const uint4 gw = lds128(at);
-            const uint32_t g4[4] = {gw.x, gw.y, gw.z, gw.w};
-            const float4 wa = __ldg(reinterpret_cast<const float4*>(p.norm_w + c0));
-            const float4 wb = __ldg(reinterpret_cast<const float4*>(p.norm_w + c0 + 4));
-            const float w8[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+            gq[j4] = lds128(st + (c0 >> 6) * 4096 + sw128(lane, (c0 & 63) >> 3));
+            wq[2 * j4] = *reinterpret_cast<const float4*>(wsm + c0);
+            wq[2 * j4 + 1] = *reinterpret_cast<const float4*>(wsm + c0 + 4);
+          }
+          tmem_wait_ld();
+          // o / rms * w * sigmoid(g), written where the gate was
+#pragma unroll
+          for (int j4 = 0; j4 < 4; ++j4) {
+            const int c0 = 32 * cb + 8 * j4;
+            const uint32_t g4[4] = {gq[j4].x, gq[j4].y, gq[j4].z, gq[j4].w};
+            const float w8[8] = {wq[2 * j4].x, wq[2 * j4].y, wq[2 * j4].z, wq[2 * j4].w,
+                                 wq[2 * j4 + 1].x, wq[2 * j4 + 1].y, wq[2 * j4 + 1].z, wq[2 * j4 + 1].w};
             uint32_t pk[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
@@ -1182,7 +1208,7 @@ __device__ __forceinline__ void state_output_loop(uint8_t* smem, uint32_t tmem, 
               pk[u] = pack_bf16(x[8 * j4 + 2 * u] * rinv * w8[2 * u] * epi::sigmoid_tanh(gv.x),
                                 x[8 * j4 + 2 * u + 1] * rinv * w8[2 * u + 1] * epi::sigmoid_tanh(gv.y));
             }
-            sts128(at, make_uint4(pk[0], pk[1], pk[2], pk[3]));
+            sts128(st + (c0 >> 6) * 4096 + sw128(lane, (c0 & 63) >> 3), make_uint4(pk[0], pk[1], pk[2], pk[3]));
           }
         }
         tc_fence_before();
@@ -1376,6 +1402,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(&bars[BS_O_FREE + 0], 64);
       mbar_init(&bars[BS_O_FREE + 1], 64);
       mbar_init(&bars[BS_FIN], 1);
+      mbar_init(&bars[BS_G_FULL + 0], 1);
+      mbar_init(&bars[BS_G_FULL + 1], 1);
     } else {
       for (int g = 0; g < LY::NGROUP; ++g) {
         uint64_t* gbars = reinterpret_cast<uint64_t*>(smem + LY::MISC + g * LY::MISC_GROUP + LY::M_BAR);
@@ -1397,6 +1425,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       sts128(smem + LY::L + sw128(rr, jj), make_uint4(pk[0], pk[1], pk[2], pk[3]));
     }
     fence_proxy_async_smem();
+  }
+  if constexpr (GATED) {
+    if (is_state && threadIdx.x < D / 4)
+      reinterpret_cast<float4*>(smem + ST_W)[threadIdx.x] = __ldg(reinterpret_cast<const float4*>(p.norm_w) + threadIdx.x);
   }
   if (warp == 0) {
     tmem_alloc(tmem_slot, 512);
