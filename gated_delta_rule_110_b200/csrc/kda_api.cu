@@ -158,10 +158,13 @@ struct PrefillPlan {
 // kTransformCost times as long per chunk as a state CTA spends on one chunk
 // of its chain.  R minimises the larger of the two times.
 constexpr double kTransformCost = 2.0;
-// A state CTA with the output epilogue fused spends about kFusedGateCost
-// times as long per chunk; the epilogue is fused where that still does not
-// make the state CTAs the bound, else it runs as a separate pass over o.
-constexpr double kFusedGateCost = 1.5;
+// The fused output epilogue keeps the state CTAs' two output warps busy for
+// about as long as a state CTA spends on a chunk, so it is free only where
+// the transform CTAs bound the call: it is fused where the transform side's
+// time exceeds the state side's by kFuseMargin, else it runs as a separate
+// pass over o.  (Measured on B200: fused wins on the 4 x 4096 and the
+// 8-sequence varlen prefills, the separate pass on one 128K-token sequence.)
+constexpr double kFuseMargin = 1.05;
 constexpr size_t kRingL2Bytes = 48u << 20;
 constexpr int kMinPreferredRing = 4;
 
@@ -193,7 +196,7 @@ PrefillPlan plan_prefill(const kda_shape& s, int64_t N, int nsm) {
   {
     const double t_state = static_cast<double>((chains + R - 1) / R);
     const double t_tf = static_cast<double>(chains) * kTransformCost / (grid - R);
-    pl.fuse_gate = t_state * kFusedGateCost <= t_tf;
+    pl.fuse_gate = t_state * kFuseMargin <= t_tf;
   }
   pl.flag_bytes = kda::pipe::flag_words(R) * sizeof(uint32_t);
   pl.ring_off = (pl.flag_bytes + 1023) & ~static_cast<size_t>(1023);

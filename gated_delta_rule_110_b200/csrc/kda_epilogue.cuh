@@ -14,16 +14,14 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include "kda_ptx.cuh"
+
 namespace kda {
 namespace epi {
 
 // sigmoid(g) = (1 + tanh(g / 2)) / 2 with the MUFU tanh (about 2^-11
 // relative error, so the sigmoid is within ~2.5e-4 absolute)
-__device__ __forceinline__ float sigmoid_tanh(float g) {
-  float t;
-  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * g));
-  return fmaf(0.5f, t, 0.5f);
-}
+__device__ __forceinline__ float sigmoid_tanh(float g) { return fmaf(0.5f, tanh_approx(0.5f * g), 0.5f); }
 
 template <typename TO>
 struct Vec8;  // 8 consecutive values of a row

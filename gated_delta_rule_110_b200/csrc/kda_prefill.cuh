@@ -1159,7 +1159,8 @@ __device__ __forceinline__ void state_output_loop(uint8_t* smem, uint32_t tmem, 
       tc_fence_after();
       if constexpr (GATED) {
         // the row's mean square (one pass over TMEM), then the products again
-        float ss0 = 0.f, ss1 = 0.f;
+        // (fp32 pairs: one packed instruction per two values)
+        uint64_t ssa = 0, ssb = 0;
 #pragma unroll 1
         for (int cb = 0; cb < 4; cb += 2) {
           float x[64];
@@ -1167,12 +1168,16 @@ __device__ __forceinline__ void state_output_loop(uint8_t* smem, uint32_t tmem, 
           tmem_ld32(tmem + lane_off + TS_O + 128 * b + 32 * cb + 32, *reinterpret_cast<float (*)[32]>(x + 32));
           tmem_wait_ld();
 #pragma unroll
-          for (int u = 0; u < 64; u += 2) {
-            ss0 = fmaf(x[u], x[u], ss0);
-            ss1 = fmaf(x[u + 1], x[u + 1], ss1);
+          for (int u = 0; u < 64; u += 4) {
+            const uint64_t xa = f2pack(x[u], x[u + 1]), xb = f2pack(x[u + 2], x[u + 3]);
+            ssa = ffma2(xa, xa, ssa);
+            ssb = ffma2(xb, xb, ssb);
           }
         }
-        const float rinv = rsqrtf((ss0 + ss1) * (1.f / D) + p.eps);
+        const float2 sa = f2unpack(ssa), sb = f2unpack(ssb);
+        const float rinv = rsqrtf(((sa.x + sa.y) + (sb.x + sb.y)) * (1.f / D) + p.eps);
+        // y = x (rinv / 2) (w + w tanh(g / 2)) = x / rms * w * sigmoid(g)
+        const uint64_t hr2 = f2pack(0.5f * rinv, 0.5f * rinv), half2 = f2pack(0.5f, 0.5f);
         if (!mbar_wait_warp(&bars[BS_G_FULL + sub], pos & 1, abort_flag)) {
           drain_tile(&bars[BS_G_FULL + sub], pos & 1);
           ok = false;
@@ -1205,8 +1210,12 @@ __device__ __forceinline__ void state_output_loop(uint8_t* smem, uint32_t tmem, 
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
               const float2 gv = bf2f(g4[u]);
-              pk[u] = pack_bf16(x[8 * j4 + 2 * u] * rinv * w8[2 * u] * epi::sigmoid_tanh(gv.x),
-                                x[8 * j4 + 2 * u + 1] * rinv * w8[2 * u + 1] * epi::sigmoid_tanh(gv.y));
+              const float2 hg = f2unpack(fmul2(f2pack(gv.x, gv.y), half2));
+              const uint64_t t2 = f2pack(tanh_approx(hg.x), tanh_approx(hg.y));
+              const uint64_t w2 = f2pack(w8[2 * u], w8[2 * u + 1]);
+              const float2 y = f2unpack(fmul2(fmul2(f2pack(x[8 * j4 + 2 * u], x[8 * j4 + 2 * u + 1]), hr2),
+                                              ffma2(w2, t2, w2)));
+              pk[u] = pack_bf16(y.x, y.y);
             }
             sts128(st + (c0 >> 6) * 4096 + sw128(lane, (c0 & 63) >> 3), make_uint4(pk[0], pk[1], pk[2], pk[3]));
           }
