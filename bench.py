@@ -353,7 +353,8 @@ def prefill_leg(kda, gen, wname, steps, warmup, world, rank, local, stream, peak
     out = {
         "value": tokens * world * steps / t, "unit": "tokens/s", "ms_per_step": ms, "steps": steps,
         "config": {"workload": f"{wname} {w.B}x{w.T} tokens H{w.H} dk=dv={w.dk} C64, bf16 q/k/v/gates, fp32 state"
-                               + (", fused per-head RMSNorm + sigmoid output gate (bf16 gate)" if gated else ""),
+                               + (", then per-head RMSNorm + sigmoid output gate (bf16 gate; fused into the prefill kernel "
+                                  "where its transform CTAs bound the call, else a separate pass over o)" if gated else ""),
                    "sequences": N, "tokens": tokens, "H": w.H,
                    "l2": f"inputs larger than L2 (no flush): {tokens * w.H * w.dk * 8 / 1e6:.0f} MB read per call"},
         "roofline": {"kernel": "kda_prefill_kernel (one cooperative launch per call)", "bound": "hbm",
@@ -429,6 +430,9 @@ def run_ours(args):
     gtd = prefill_leg(kda, gen, "prefill", args.steps, args.warmup, world, rank, local, stream, peaks, peak_src,
                       counters, gated=True)
     launches += args.steps
+    vgt = prefill_leg(kda, gen, "varlen", args.steps, args.warmup, world, rank, local, stream, peaks, peak_src,
+                      counters, gated=True)
+    launches += args.steps
     lgt = prefill_leg(kda, gen, "long", long_steps, args.warmup, world, rank, local, stream, peaks, peak_src,
                       counters, gated=True)
     launches += 2 * long_steps  # the prefill kernel and the separate epilogue pass
@@ -482,6 +486,7 @@ def run_ours(args):
             "varlen": var,
             "long": lng,
             "prefill_gated": gtd,
+            "varlen_gated": vgt,
             "long_gated": lgt,
             "decode": {"value": world * dec_steps / t_dec, "unit": "steps/s", "ms_per_step": dec_ms,
                        "steps": dec_steps,
