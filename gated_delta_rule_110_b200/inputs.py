@@ -33,6 +33,8 @@ from __future__ import annotations
 
 from dataclasses import dataclass, field
 
+import math
+
 import torch
 
 
@@ -150,6 +152,36 @@ def output_gate_inputs(v_shape, *, dtype=torch.bfloat16, scale: float = 2.0, see
     gate = (scale * _normal(tuple(v_shape), g, device)).to(dtype)
     w = 0.5 + torch.rand((v_shape[-1],), generator=g, device=device)
     return gate, w
+
+
+def make_layer_inputs(B: int, T: int, H: int, dk: int, dv: int, *, dtype=torch.bfloat16, seqlens=None,
+                      seed: int = 0, device="cpu") -> dict:
+    """Inputs of the operator with the layer's producer steps: raw q, k
+    (normal, not normalised; each row scaled by U(0.5, 2)), v, the decay
+    gate's projection output f ~ N(0, 1) (dtype), per-head A_log = log A with
+    A ~ U(1, 16) and per-(head, channel) dt_bias = softplus^-1(dt) with
+    log dt ~ U(log 1e-3, log 1e-1) (fp32, Mamba's initialisation ranges),
+    beta, S0 and cu_seqlens as make_inputs."""
+    g = torch.Generator(device=device).manual_seed(seed)
+    N = len(seqlens) if seqlens is not None else B
+    if seqlens is not None and (B != 1 or T != sum(seqlens)):
+        raise ValueError("packed inputs need B == 1 and T == sum(seqlens)")
+    q = _normal((B, T, H, dk), g, device) * (0.5 + 1.5 * torch.rand((B, T, H, 1), generator=g, device=device))
+    k = _normal((B, T, H, dk), g, device) * (0.5 + 1.5 * torch.rand((B, T, H, 1), generator=g, device=device))
+    v = _normal((B, T, H, dv), g, device)
+    f = _normal((B, T, H, dk), g, device)
+    A_log = torch.log(1.0 + 15.0 * torch.rand((H,), generator=g, device=device))
+    dt = torch.exp(math.log(1e-3) + (math.log(1e-1) - math.log(1e-3)) * torch.rand((H, dk), generator=g, device=device))
+    dt_bias = dt + torch.log(-torch.expm1(-dt))
+    beta = torch.sigmoid(_normal((B, T, H), g, device))
+    S0 = 0.1 * _normal((N, H, dk, dv), g, device)
+    cu = None
+    if seqlens is not None:
+        cu = torch.zeros(N + 1, dtype=torch.int32)
+        cu[1:] = torch.cumsum(torch.tensor(seqlens, dtype=torch.int64), 0).to(torch.int32)
+        cu = cu.to(device)
+    return dict(q=q.to(dtype), k=k.to(dtype), v=v.to(dtype), f=f.to(dtype), A_log=A_log, dt_bias=dt_bias,
+                beta=beta.to(dtype), S0=S0, cu_seqlens=cu)
 
 
 def workload_inputs(w: Workload, device="cpu", seed_offset: int = 0) -> dict:

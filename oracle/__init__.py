@@ -53,6 +53,10 @@ def _load():
         lib.kda_oracle_mutation_count.restype = ctypes.c_int
         lib.kda_oracle_output_gate.argtypes = [ctypes.c_int64, ctypes.c_int, dp, dp, dp, ctypes.c_double, dp]
         lib.kda_oracle_output_gate.restype = ctypes.c_int
+        lib.kda_oracle_l2norm.argtypes = [ctypes.c_int64, ctypes.c_int, dp, ctypes.c_double, dp]
+        lib.kda_oracle_l2norm.restype = ctypes.c_int
+        lib.kda_oracle_decay_gate.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, dp, dp, dp, dp]
+        lib.kda_oracle_decay_gate.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -130,3 +134,40 @@ def output_gate(o, g, w, eps: float):
     if rc != 0:
         raise ValueError("oracle rejected its arguments")
     return out
+
+
+def l2norm(x, eps: float):
+    """x / sqrt(sum(x^2) + eps) over the last axis, in fp64 (the L2
+    normalisation of q and k); returns an array shaped like x."""
+    x = _f64(x)
+    d = x.shape[-1]
+    out = np.zeros_like(x)
+    if _load().kda_oracle_l2norm(x.size // d, d, _ptr(x), float(eps), _ptr(out)) != 0:
+        raise ValueError("oracle rejected its arguments")
+    return out
+
+
+def decay_gate(f, A_log, dt_bias):
+    """log alpha = -exp(A_log[h]) * softplus(f + dt_bias[h, c]) in fp64.
+    f: [..., H, dk]; A_log: [H]; dt_bias: [H, dk]."""
+    f, A_log, dt_bias = _f64(f), _f64(A_log), _f64(dt_bias)
+    H, dk = f.shape[-2], f.shape[-1]
+    if A_log.shape != (H,) or dt_bias.shape != (H, dk):
+        raise ValueError("A_log must be [H] and dt_bias [H, dk]")
+    out = np.zeros_like(f)
+    if _load().kda_oracle_decay_gate(f.size // (H * dk), H, dk, _ptr(f), _ptr(A_log), _ptr(dt_bias), _ptr(out)) != 0:
+        raise ValueError("oracle rejected its arguments")
+    return out
+
+
+def forward_layer(q, k, v, f, A_log, dt_bias, beta, S0=None, cu_seqlens=None, qk_eps: float = 1e-6,
+                  out_gate=None, norm_weight=None, eps: float = 1e-5):
+    """The operator with the layer's producer and (optionally) consumer steps,
+    composed from the functions above: forward(l2norm(q), l2norm(k), v,
+    decay_gate(f, A_log, dt_bias), beta, S0), then output_gate when out_gate
+    is given.  Returns (o, S_T)."""
+    o, S = forward(l2norm(q, qk_eps), l2norm(k, qk_eps), v, decay_gate(f, A_log, dt_bias), beta, S0,
+                   cu_seqlens=cu_seqlens)
+    if out_gate is not None:
+        o = output_gate(o, out_gate, norm_weight, eps)
+    return o, S

@@ -271,3 +271,52 @@ int kda_oracle_output_gate(int64_t rows, int dv, const double* o, const double* 
   }
   return 0;
 }
+
+/*
+ * kda_oracle_l2norm -- the L2 normalisation of the query and the key that the
+ * "Kimi Linear" summary (section "Configuração do modelo Kimi Linear") adds
+ * for the stability of the transition's eigenvalues.  Per row (one token and
+ * head) of d values:
+ *
+ *     out[j] = x[j] / sqrt( sum_i x[i]^2 + eps )
+ *
+ * eps >= 0 keeps a zero row at zero (the page names no epsilon).
+ */
+int kda_oracle_l2norm(int64_t rows, int d, const double* x, double eps, double* out) {
+  if (rows < 0 || d <= 0 || !x || !out || !(eps >= 0.0)) return -1;
+  for (int64_t r = 0; r < rows; ++r) {
+    double ss = 0.0;
+    for (int j = 0; j < d; ++j) ss += x[r * d + j] * x[r * d + j];
+    const double n = sqrt(ss + eps);
+    for (int j = 0; j < d; ++j) out[r * d + j] = n > 0.0 ? x[r * d + j] / n : 0.0;
+  }
+  return 0;
+}
+
+/* log(1 + e^x) without overflow */
+static double softplus(double x) { return x > 0.0 ? x + log1p(exp(-x)) : log1p(exp(x)); }
+
+/*
+ * kda_oracle_decay_gate -- the channel-wise decay gate.  The same page
+ * parametrises it by a low-rank projection (its output f, one value per key
+ * channel) and a decay function "like GDN's and Mamba's": a positive step
+ * size softplus(f + bias) times a negative per-head rate -exp(A_log).  Per
+ * token t, head h, channel c:
+ *
+ *     log alpha[t][h][c] = -exp(A_log[h]) * softplus(f[t][h][c] + dt_bias[h][c])
+ *
+ * f, out: [tokens, H, dk]; A_log: [H]; dt_bias: [H, dk].
+ */
+int kda_oracle_decay_gate(int64_t tokens, int H, int dk, const double* f, const double* A_log,
+                          const double* dt_bias, double* out) {
+  if (tokens < 0 || H <= 0 || dk <= 0 || !f || !A_log || !dt_bias || !out) return -1;
+  for (int64_t t = 0; t < tokens; ++t)
+    for (int h = 0; h < H; ++h) {
+      const double rate = exp(A_log[h]);
+      for (int c = 0; c < dk; ++c) {
+        const int64_t e = (t * H + h) * dk + c;
+        out[e] = -rate * softplus(f[e] + dt_bias[h * dk + c]);
+      }
+    }
+  return 0;
+}
