@@ -12,6 +12,8 @@ Entry points (same names as the C ABI):
   chunkwise-parallel prefill -> ``(o, S_T)``
 * ``kda_decode_step(q, k, v, log_alpha, beta, S)`` one recurrent token per
   (sequence, head), ``S`` updated in place -> ``o``
+* ``kda_chunk_fwd_layer(q, k, v, gate_f, A_log, dt_bias, beta, ...)`` raw q, k and
+  the decay gate's projection in (L2 norm and gate computed in the kernel) -> ``(o, S_T)``
 * ``kda_chunk_fwd_gated(q, k, v, log_alpha, beta, out_gate, norm_weight, ...)``
   prefill with the per-head RMSNorm and sigmoid output gate fused -> ``(o', S_T)``
 * ``kda_chunk_fwd_slots(q, k, v, log_alpha, beta, state_pool, state_slots,
@@ -45,7 +47,8 @@ _STATUS_NAMES = {
 }
 
 EXPORTED_SYMBOLS = (
-    "kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_chunk_fwd_gated", "kda_chunk_fwd_noalloc",
+    "kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_chunk_fwd_gated", "kda_chunk_fwd_layer",
+    "kda_chunk_fwd_noalloc",
     "kda_chunk_fwd_slots",
     "kda_decode_step", "kda_decode_step_slots", "kda_check_device_error", "kda_status_string",
     "kda_abi_version",
@@ -93,6 +96,9 @@ def load_library(build_if_missing: bool = True):
     lib.kda_chunk_fwd_gated.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp, vp,
                                         ctypes.c_size_t, vp]
     lib.kda_chunk_fwd_gated.restype = ctypes.c_int
+    lib.kda_chunk_fwd_layer.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp, vp,
+                                        ctypes.c_size_t, vp]
+    lib.kda_chunk_fwd_layer.restype = ctypes.c_int
     lib.kda_chunk_fwd_noalloc.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.kda_chunk_fwd_noalloc.restype = ctypes.c_int
     lib.kda_chunk_fwd_slots.argtypes = [sp, vp, vp, vp, vp, vp, vp, ctypes.c_int32, vp, vp, vp, vp, vp,
@@ -237,6 +243,50 @@ def kda_chunk_fwd_gated(q, k, v, log_alpha, beta, out_gate, norm_weight, S0=None
         _stream(stream))
     if rc != KDA_OK:
         raise KdaError(rc, "kda_chunk_fwd_gated")
+    return o, S_T
+
+
+def kda_chunk_fwd_layer(q, k, v, gate_f, A_log, dt_bias, beta, S0=None, cu_seqlens=None, *, out_gate=None,
+                        norm_weight=None, eps: float = 1e-5, chunk: int = 64, o=None, S_T=None, workspace=None,
+                        stream=None, validate: bool = False, output_final_state: bool = True,
+                        gate_mode: str = "auto", state_ctas: int = 0, grid_ctas: int = 0):
+    """The operator with the Kimi Linear layer's producer steps fused (raw q,
+    k are L2-normalised, log alpha = -exp(A_log) * softplus(gate_f + dt_bias))
+    and, with ``out_gate`` / ``norm_weight``, its output epilogue
+    (include/kda.h, kda_chunk_fwd_layer).  Returns (o, S_T)."""
+    import torch
+    _need_cuda(q, k, v, gate_f, A_log, dt_bias, beta, S0, cu_seqlens, out_gate, norm_weight, o, S_T, workspace)
+    H, dk = q.shape[2], q.shape[3]
+    if gate_f.shape != q.shape or gate_f.dtype != q.dtype:
+        raise ValueError("gate_f must have the shape and dtype of q")
+    if A_log.dtype != torch.float32 or A_log.numel() != H or dt_bias.dtype != torch.float32 or dt_bias.numel() != H * dk:
+        raise ValueError("A_log must be float32 [H] and dt_bias float32 [H, dk]")
+    if (out_gate is None) != (norm_weight is None):
+        raise ValueError("out_gate and norm_weight go together")
+    if out_gate is not None:
+        if out_gate.shape != v.shape or out_gate.dtype != v.dtype:
+            raise ValueError("out_gate must have the shape and dtype of v")
+        if norm_weight.dtype != torch.float32 or norm_weight.numel() != v.shape[-1]:
+            raise ValueError("norm_weight must be a float32 tensor of dv values")
+    if gate_mode not in _GATE_MODES:
+        raise ValueError(f"gate_mode must be one of {sorted(_GATE_MODES)}")
+    shape = _shape_of(q, v, gate_f, cu_seqlens, chunk, validate, False, state_ctas, grid_ctas)
+    shape.flags |= _GATE_MODES[gate_mode]
+    N = shape.B if cu_seqlens is None else shape.n_seqs
+    if o is None:
+        o = torch.empty(v.shape, dtype=v.dtype, device=v.device)
+    if S_T is None and output_final_state:
+        S_T = torch.empty((N, shape.H, shape.dk, shape.dv), dtype=torch.float32, device=q.device)
+    need = kda_chunk_fwd_workspace_size(shape)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = load_library().kda_chunk_fwd_layer(
+        ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(gate_f), _ptr(A_log), _ptr(dt_bias), _ptr(beta),
+        _ptr(S0), _ptr(cu_seqlens), _ptr(out_gate), _ptr(norm_weight), float(eps), _ptr(o), _ptr(S_T),
+        _ptr(workspace), ws_bytes, _stream(stream))
+    if rc != KDA_OK:
+        raise KdaError(rc, "kda_chunk_fwd_layer")
     return o, S_T
 
 

@@ -134,6 +134,14 @@ struct Epilogue {
   float eps = 0.f;
 };
 
+// Optional producer steps of the tensor-core prefill (A_log == nullptr: none):
+// q, k are L2-normalised in the kernel and log_alpha carries the decay gate's
+// projection f, log alpha = -exp(A_log[h]) * softplus(f + dt_bias[h][c]).
+struct Producer {
+  const float* A_log = nullptr;
+  const float* dt_bias = nullptr;
+};
+
 struct PrefillPlan {
   int R = 0;             // state CTAs
   bool fuse_gate = false;  // output epilogue in the state CTAs (they have time to spare)
@@ -214,10 +222,10 @@ PrefillPlan plan_prefill(const kda_shape& s, int64_t N, int nsm) {
 
 // With an epilogue, *fused says whether the kernel applied it (else the caller
 // runs the separate pass).
-template <typename TG>
+template <typename TG, bool PROD>
 kda_status launch_prefill(const kda_shape& s, int64_t N, int64_t Ttot, const void* q, const void* k, const void* v,
                           const void* la, const void* beta, const kda::StateIO& io, const Epilogue& ep_req,
-                          const int32_t* cu, void* o,
+                          const Producer& pr, const int32_t* cu, void* o,
                           void* ws, size_t ws_bytes, cudaStream_t st, bool* fused) {
   namespace P = kda::pipe;
   const PrefillPlan pl = plan_prefill(s, N, device_sm_count());
@@ -255,12 +263,14 @@ kda_status launch_prefill(const kda_shape& s, int64_t N, int64_t Ttot, const voi
   prm.beta = beta;
   prm.st = io;
   prm.o = static_cast<__nv_bfloat16*>(o);
+  prm.A_log = pr.A_log;
+  prm.dt_bias = pr.dt_bias;
   prm.gate = static_cast<const __nv_bfloat16*>(ep.gate);
   prm.norm_w = ep.norm_w;
   prm.eps = ep.eps;
   prm.flags = static_cast<uint32_t*>(ws);
   prm.ring = static_cast<uint8_t*>(ws) + pl.ring_off;
-  auto* kern = ep.gate ? P::kda_prefill_kernel<TG, true> : P::kda_prefill_kernel<TG, false>;
+  auto* kern = ep.gate ? P::kda_prefill_kernel<TG, true, PROD> : P::kda_prefill_kernel<TG, false, PROD>;
   const uint32_t smem = P::ST_BYTES > P::TfLayout<TG>::BYTES ? P::ST_BYTES : P::TfLayout<TG>::BYTES;
   if (!ensure_smem(kern, smem)) return KDA_ERR_CUDA;
   if (cudaMemsetAsync(ws, 0, pl.flag_bytes, st) != cudaSuccess) return KDA_ERR_CUDA;
@@ -339,7 +349,8 @@ size_t kda_chunk_fwd_min_workspace(const kda_shape* sp) {
 // Shared body of kda_chunk_fwd and kda_chunk_fwd_slots; `io` says where the
 // states live (dense rows or pool slots).
 kda_status chunk_fwd(const kda_shape* sp, const void* q, const void* k, const void* v, const void* log_alpha,
-                     const void* beta, const kda::StateIO& io, const Epilogue& ep, const int32_t* cu_seqlens,
+                     const void* beta, const kda::StateIO& io, const Epilogue& ep, const Producer& pr,
+                     const int32_t* cu_seqlens,
                      void* o, void* workspace,
                      size_t workspace_bytes, void* stream) {
   kda_status e = check_common(sp);
@@ -363,15 +374,22 @@ kda_status chunk_fwd(const kda_shape* sp, const void* q, const void* k, const vo
 
   if (ep.gate && Ttot > 0 && (!aligned16(o) || !aligned16(ep.gate))) return KDA_ERR_ALIGN;
   bool fused = false;
-  if (use_tc(s) && Ttot > 0) {
+  if (pr.A_log && (!use_tc(s) || s.gate_dtype != KDA_BF16)) return KDA_ERR_UNSUPPORTED;
+  if (pr.A_log && Ttot > 0) {
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(log_alpha) || !aligned16(o) ||
+        !aligned16(pr.dt_bias))
+      return KDA_ERR_ALIGN;
+    e = launch_prefill<__nv_bfloat16, true>(s, N, Ttot, q, k, v, log_alpha, beta, io, ep, pr, cu_seqlens, o,
+                                            workspace, workspace_bytes, st, &fused);
+  } else if (use_tc(s) && Ttot > 0) {
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(log_alpha) || !aligned16(o))
       return KDA_ERR_ALIGN;
     if (s.gate_dtype == KDA_BF16)
-      e = launch_prefill<__nv_bfloat16>(s, N, Ttot, q, k, v, log_alpha, beta, io, ep, cu_seqlens, o, workspace,
-                                        workspace_bytes, st, &fused);
+      e = launch_prefill<__nv_bfloat16, false>(s, N, Ttot, q, k, v, log_alpha, beta, io, ep, pr, cu_seqlens, o,
+                                               workspace, workspace_bytes, st, &fused);
     else
-      e = launch_prefill<float>(s, N, Ttot, q, k, v, log_alpha, beta, io, ep, cu_seqlens, o, workspace,
-                                workspace_bytes, st, &fused);
+      e = launch_prefill<float, false>(s, N, Ttot, q, k, v, log_alpha, beta, io, ep, pr, cu_seqlens, o, workspace,
+                                       workspace_bytes, st, &fused);
   } else if (s.io_dtype == KDA_F32) {
     if (s.gate_dtype == KDA_F32)
       e = dispatch_recurrent_fwd<float, float>(s, N, q, k, v, log_alpha, beta, io, cu_seqlens, o, st);
@@ -423,8 +441,8 @@ kda_status kda_chunk_fwd(const kda_shape* sp, const void* q, const void* k, cons
   kda::StateIO io;
   io.S0 = S0;
   io.S_T = S_T;
-  return chunk_fwd(sp, q, k, v, log_alpha, beta, io, Epilogue{}, cu_seqlens, o, workspace, workspace_bytes,
-                   stream);
+  return chunk_fwd(sp, q, k, v, log_alpha, beta, io, Epilogue{}, Producer{}, cu_seqlens, o, workspace,
+                   workspace_bytes, stream);
 }
 
 kda_status kda_chunk_fwd_slots(const kda_shape* sp, const void* q, const void* k, const void* v,
@@ -441,8 +459,8 @@ kda_status kda_chunk_fwd_slots(const kda_shape* sp, const void* q, const void* k
   io.slots = state_slots;
   io.has_init = has_initial_state;
   io.num_slots = num_slots;
-  return chunk_fwd(sp, q, k, v, log_alpha, beta, io, Epilogue{}, cu_seqlens, o, workspace, workspace_bytes,
-                   stream);
+  return chunk_fwd(sp, q, k, v, log_alpha, beta, io, Epilogue{}, Producer{}, cu_seqlens, o, workspace,
+                   workspace_bytes, stream);
 }
 
 kda_status kda_chunk_fwd_gated(const kda_shape* sp, const void* q, const void* k, const void* v,
@@ -460,7 +478,33 @@ kda_status kda_chunk_fwd_gated(const kda_shape* sp, const void* q, const void* k
   ep.gate = out_gate;
   ep.norm_w = norm_weight;
   ep.eps = eps;
-  return chunk_fwd(sp, q, k, v, log_alpha, beta, io, ep, cu_seqlens, o, workspace, workspace_bytes, stream);
+  return chunk_fwd(sp, q, k, v, log_alpha, beta, io, ep, Producer{}, cu_seqlens, o, workspace, workspace_bytes,
+                   stream);
+}
+
+kda_status kda_chunk_fwd_layer(const kda_shape* sp, const void* q, const void* k, const void* v, const void* gate_f,
+                               const float* A_log, const float* dt_bias, const void* beta, const float* S0,
+                               const int32_t* cu_seqlens, const void* out_gate, const float* norm_weight, float eps,
+                               void* o, float* S_T, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!sp) return KDA_ERR_NULL;
+  if (!A_log || !dt_bias) return KDA_ERR_NULL;
+  if (!aligned(A_log, 4) || !aligned16(dt_bias)) return KDA_ERR_ALIGN;
+  Epilogue ep;
+  if (out_gate || norm_weight) {
+    if (!out_gate || !norm_weight) return KDA_ERR_NULL;
+    if (!(eps >= 0.f) || !(eps < 3.0e38f)) return KDA_ERR_ARGUMENT;
+    if (!aligned16(out_gate) || !aligned16(norm_weight)) return KDA_ERR_ALIGN;
+    ep.gate = out_gate;
+    ep.norm_w = norm_weight;
+    ep.eps = eps;
+  }
+  kda::StateIO io;
+  io.S0 = S0;
+  io.S_T = S_T;
+  Producer pr;
+  pr.A_log = A_log;
+  pr.dt_bias = dt_bias;
+  return chunk_fwd(sp, q, k, v, gate_f, beta, io, ep, pr, cu_seqlens, o, workspace, workspace_bytes, stream);
 }
 
 kda_status kda_decode_step(const kda_shape* sp, const void* q, const void* k, const void* v, const void* log_alpha,

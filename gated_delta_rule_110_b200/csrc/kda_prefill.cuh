@@ -63,6 +63,7 @@ constexpr int NTHREADS = 384;
 constexpr int MAX_RING = 16;  // ring slots per state CTA (the host picks 2..16)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kSpan2 = 230.0f;  // largest chunk decay of the factorised path, log2 units
+constexpr float kQKNormEps = 1e-6f;  // epsilon of the producer's L2 normalisation of q and k
 
 // ---- ring slot: operands of one chunk as the state CTA's MMAs read them ----
 // Part A (Tb, -W'^T, the per-channel scales) feeds U and is released once U
@@ -154,6 +155,11 @@ struct Params {
   const void* beta;
   StateIO st;       // initial / final states (dense rows or pool slots)
   __nv_bfloat16* o;
+  // producer steps (PROD instantiation): q, k are raw and L2-normalised here;
+  // the log-decay tile is the gate projection f, log alpha = -exp(A_log[h]) *
+  // softplus(f + dt_bias[h][c])
+  const float* A_log;    // [H]
+  const float* dt_bias;  // [H][dk]
   // optional output epilogue (gate == nullptr: o is written as computed):
   // o <- o / rms(o) * norm_w * sigmoid(gate), rms over the head's dv values
   const __nv_bfloat16* gate;  // [B, T, H, dv], like o
@@ -237,8 +243,10 @@ __device__ __forceinline__ int swzA(int r, int s) { return r * 64 + (s ^ ((((r &
 
 // ===========================================================================
 // transform role: one group of 4 compute warps + a load warp + an MMA warp
+// PROD: the producer steps (L2 norm of q and k, the decay gate from its
+// projection) run here, on the raw tiles; TG is then bf16.
 // ===========================================================================
-template <typename TG>
+template <typename TG, bool PROD>
 struct Tf {
   using LY = TfLayout<TG>;
   uint8_t* smem;
@@ -270,10 +278,15 @@ struct Tf {
   }
   __device__ static int tcol(int r, int s) { return s ^ ((((r & 7) ^ ((r >> 3) & 7))) << 2); }
   __device__ float* amat() const { return reinterpret_cast<float*>(gb + LY::G_KB); }
+  // producer: 1/|q_r| at [r], 1/|k_r| at [64 + r] (the upper half of the
+  // log-decay tile is dead from the cumsum MMA until the next raw tiles)
+  __device__ float* qk_norms() const { return reinterpret_cast<float*>(gb + LY::G_RL + 10240); }
   __device__ void bar() const { named_bar(1 + g, 128); }
   // The cumsum operand is the raw TMA tile unless rows past the chunk end must
-  // be zeroed or fp32 gates must be split into bf16 parts first.
-  __device__ static bool needs_prep(int L) { return sizeof(TG) != 2 || L < C; }
+  // be zeroed, or fp32 gates (or the producer's log-decay) must be split into
+  // bf16 parts first.
+  __device__ static bool needs_prep(int L) { return PROD || sizeof(TG) != 2 || L < C; }
+  static constexpr bool kSplitGate = PROD || sizeof(TG) != 2;
 
   // ------------------------------------------------------------ load warp
   __device__ void load_loop(const Maps& maps, const Params& p, int maxlen, volatile int* abort_flag) {
@@ -368,7 +381,10 @@ struct Tf {
         meta[MT_T0LO] = static_cast<int>(static_cast<uint64_t>(t0) & 0xffffffffu);
         meta[MT_T0HI] = static_cast<int>(static_cast<uint64_t>(t0) >> 32);
         const int y = static_cast<int>(t0);
-        mbar_arrive_expect_tx(&bars[BT_RAW_FULL], 32768 + LY::RL_BYTES);
+        mbar_arrive_expect_tx(&bars[BT_RAW_FULL], 32768 + LY::RL_BYTES + (PROD ? 4 * D : 0));
+        // producer: the head's dt_bias row goes where g_last lives later (dead
+        // from the previous chunk's C2 on: the raw tiles were released after it)
+        if (PROD) bulk_g2s(misc + LY::M_GL, p.dt_bias + static_cast<int64_t>(h) * D, 4 * D, &bars[BT_RAW_FULL]);
         for (int hf = 0; hf < 2; ++hf) {
           tma_load_2d(gb + LY::G_RQ + hf * 8192, &maps.q, h * D + 64 * hf, y, &bars[BT_RAW_FULL]);
           tma_load_2d(gb + LY::G_RK + hf * 8192, &maps.k, h * D + 64 * hf, y, &bars[BT_RAW_FULL]);
@@ -412,15 +428,16 @@ struct Tf {
         ++nprep;
       }
       tc_fence_after();
-      if (sizeof(TG) == 2) {
+      if (!kSplitGate) {
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           mma_bf16_ss(tmem + TT_G, make_sdesc_sw128(Lb + kk * 32, 16, 1024),
                       make_sdesc_sw128(gba + LY::G_RL + kk * 2048, 8192, 1024), id_cs, kk > 0);
       } else {
-        // log-decay split into three bf16 parts (in the KQ and KB areas)
+        // log-decay split into bf16 parts (in the KQ and KB areas): three for
+        // fp32 gates, two for the producer's (16 significant bits)
 #pragma unroll
-        for (int t = 0; t < 3; ++t) {
+        for (int t = 0; t < (PROD ? 2 : 3); ++t) {
           const uint32_t base = gba + (t < 2 ? LY::G_KQ + 16384 * t : LY::G_KB);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
@@ -498,6 +515,36 @@ struct Tf {
 
       // ---- C1: prepare the cumsum operand (when the raw tile is not usable) ----
       if (!needs_prep(L)) {
+      } else if (PROD) {
+        // log alpha = -exp(A_log[h]) * softplus(f + dt_bias[h][c]) in fp32 from
+        // the bf16 tile of f: softplus(x) = ln 2 * log2(1 + 2^(x log2 e)) on the
+        // MUFU unit (x itself beyond 15); split into hi + lo bf16 tiles
+        const float nrate = -__expf(p.A_log[hh]);
+        const float nrate_ln2 = nrate * 0.69314718f;
+        const float* bias = sgl;  // this head's dt_bias, staged by the load warp
+#pragma unroll 2
+        for (int jj = 0; jj < 8; ++jj) {
+          const int c0 = 64 * ch + 8 * jj;
+          const uint4 w = lds128(gb + LY::G_RL + ch * 8192 + sw128(r, jj));
+          const uint32_t f4[4] = {w.x, w.y, w.z, w.w};
+          const float4 ba = *reinterpret_cast<const float4*>(bias + c0);
+          const float4 bb = *reinterpret_cast<const float4*>(bias + c0 + 4);
+          const float b8[8] = {ba.x, ba.y, ba.z, ba.w, bb.x, bb.y, bb.z, bb.w};
+          uint32_t pk[2][4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float2 fx = bf2f(f4[u]);
+            const float x0 = fx.x + b8[2 * u], x1 = fx.y + b8[2 * u + 1];
+            float a0 = x0 > 15.f ? nrate * x0 : nrate_ln2 * lg2_approx(1.f + ex2_approx(x0 * kLog2e));
+            float a1 = x1 > 15.f ? nrate * x1 : nrate_ln2 * lg2_approx(1.f + ex2_approx(x1 * kLog2e));
+            if (r >= L) a0 = a1 = 0.f;
+            const float h0 = __bfloat162float(__float2bfloat16_rn(a0)), h1 = __bfloat162float(__float2bfloat16_rn(a1));
+            pk[0][u] = pack_bf16(h0, h1);
+            pk[1][u] = pack_bf16(a0 - h0, a1 - h1);
+          }
+          sts128(gb + LY::G_KQ + ch * 8192 + sw128(r, jj), make_uint4(pk[0][0], pk[0][1], pk[0][2], pk[0][3]));
+          sts128(gb + LY::G_KQ + 16384 + ch * 8192 + sw128(r, jj), make_uint4(pk[1][0], pk[1][1], pk[1][2], pk[1][3]));
+        }
       } else if (sizeof(TG) == 2) {
         if (L < C) {
           for (int e = gt; e < (C - L) * 16; e += 128) {
@@ -546,6 +593,25 @@ struct Tf {
 
       // ---- C2: cumulative decay -> scaled tiles ---------------------------------
       if (gt < C) sbeta[gt] = beta_r;  // published by the barriers below
+      // producer: |q_r|^2 and |k_r|^2 over this thread's channel half while the
+      // cumsum MMA runs; the halves meet in the upper half of the log-decay
+      // tile (consumed by C1), read after the barriers below
+      float sq = 0.f, sk = 0.f;
+      if constexpr (PROD) {
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          const uint4 kw = lds128(gb + LY::G_RK + ch * 8192 + sw128(r, jj));
+          const uint4 qw = lds128(gb + LY::G_RQ + ch * 8192 + sw128(r, jj));
+          const uint32_t kk4[4] = {kw.x, kw.y, kw.z, kw.w}, qq4[4] = {qw.x, qw.y, qw.z, qw.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float2 kx = bf2f(kk4[u]), qx = bf2f(qq4[u]);
+            sk = fmaf(kx.x, kx.x, fmaf(kx.y, kx.y, sk));
+            sq = fmaf(qx.x, qx.x, fmaf(qx.y, qx.y, sq));
+          }
+        }
+        reinterpret_cast<float2*>(gb + LY::G_RL + 9216)[ch * 64 + r] = make_float2(sq, sk);
+      }
       mbar_wait_warp(&bars[BT_CS_FULL], it & 1, abort_flag);
       tc_fence_after();
       float g2[64];
@@ -579,6 +645,19 @@ struct Tf {
         vec[128 + gt] = ex2_approx(gl);
       }
       bar();
+      // producer: 1 / |q_r| and 1 / |k_r| from both halves' partial sums; the
+      // exact path reads every row's factors (published by its own barrier)
+      float rq = 1.f, rk = 1.f;
+      if constexpr (PROD) {
+        const float2 o = reinterpret_cast<const float2*>(gb + LY::G_RL + 9216)[(ch ^ 1) * 64 + r];
+        rq = rsqrtf(sq + o.x + kQKNormEps);
+        rk = rsqrtf(sk + o.y + kQKNormEps);
+        if (ch == 0) {
+          float* rn = qk_norms();
+          rn[r] = rq;
+          rn[64 + r] = rk;
+        }
+      }
       // q_r . k_r over this thread's channel half, in fp32 from the raw bf16
       // inputs: the diagonal of P, where the decay factors cancel exactly.  The
       // bf16-rounded scaled operands would lose it to cancellation when q_r and
@@ -603,7 +682,11 @@ struct Tf {
           uint32_t ka[4], qa[4], kb[4], kt[4];
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            const float2 kx = bf2f(kk4[u]), qx = bf2f(qq4[u]);
+            float2 kx = bf2f(kk4[u]), qx = bf2f(qq4[u]);
+            if constexpr (PROD) {
+              kx.x *= rk, kx.y *= rk;
+              qx.x *= rq, qx.y *= rq;
+            }
             pdiag = fmaf(qx.x, kx.x, fmaf(qx.y, kx.y, pdiag));
             const float rf0 = rf8[2 * u], rf1 = rf8[2 * u + 1];
             const float x0 = g2[8 * jj + 2 * u], x1 = g2[8 * jj + 2 * u + 1];
@@ -655,6 +738,11 @@ struct Tf {
               pp += kval(RQ, ar, c) * kse;
             }
           }
+          if constexpr (PROD) {
+            const float* rn = qk_norms();
+            a *= rn[64 + ar] * rn[64 + as];
+            pp *= rn[ar] * rn[64 + as];
+          }
           Af[swzA(ar, as)] = as < ar ? sbeta[ar] * a : 0.f;
           *reinterpret_cast<__nv_bfloat16*>(gb + LY::G_RL + sw128(ar, as >> 3) + (as & 7) * 2) =
               __float2bfloat16_rn(pp);
@@ -671,7 +759,11 @@ struct Tf {
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             const int c = c0 + 2 * u;
-            const float2 kx = bf2f(kk4[u]), qx = bf2f(qq4[u]);
+            float2 kx = bf2f(kk4[u]), qx = bf2f(qq4[u]);
+            if constexpr (PROD) {
+              kx.x *= rk, kx.y *= rk;
+              qx.x *= rq, qx.y *= rq;
+            }
             const float x0 = g2[8 * jj + 2 * u], x1 = g2[8 * jj + 2 * u + 1];
             const float gm0 = ex2_approx(x0), gm1 = ex2_approx(x1);
             const float ps0 = ex2_approx(sgl[c] - x0), ps1 = ex2_approx(sgl[c + 1] - x1);
@@ -1368,7 +1460,7 @@ __device__ __forceinline__ void state_warps_loop(uint8_t* smem, uint32_t tmem, c
 // ===========================================================================
 // the kernel
 // ===========================================================================
-template <typename TG, bool GATED>
+template <typename TG, bool GATED, bool PROD>
 __global__ void __launch_bounds__(NTHREADS, 1)
     kda_prefill_kernel(const __grid_constant__ Maps maps, const Params p) {
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -1465,7 +1557,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   } else {
     const int g = (warp < 8) ? (warp >> 2) : ((warp - 8) & 1);
     if (g < LY::NGROUP) {
-      Tf<TG> tf(smem, tmem, g);
+      Tf<TG, PROD> tf(smem, tmem, g);
       if (warp < 8) {
         tf.compute_loop(p, abort_flag);
       } else if (warp < 10) {

@@ -403,6 +403,13 @@ __device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
   return d;
 }
 
+// log2(x) on the MUFU unit (approximate, flush-to-zero).
+__device__ __forceinline__ float lg2_approx(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // 2^x on the MUFU unit (approximate, flush-to-zero).
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;

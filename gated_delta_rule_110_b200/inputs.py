@@ -155,13 +155,15 @@ def output_gate_inputs(v_shape, *, dtype=torch.bfloat16, scale: float = 2.0, see
 
 
 def make_layer_inputs(B: int, T: int, H: int, dk: int, dv: int, *, dtype=torch.bfloat16, seqlens=None,
-                      seed: int = 0, device="cpu") -> dict:
+                      seed: int = 0, device="cpu", dt_range=(1e-3, 1e-1)) -> dict:
     """Inputs of the operator with the layer's producer steps: raw q, k
     (normal, not normalised; each row scaled by U(0.5, 2)), v, the decay
     gate's projection output f ~ N(0, 1) (dtype), per-head A_log = log A with
     A ~ U(1, 16) and per-(head, channel) dt_bias = softplus^-1(dt) with
-    log dt ~ U(log 1e-3, log 1e-1) (fp32, Mamba's initialisation ranges),
-    beta, S0 and cu_seqlens as make_inputs."""
+    log dt ~ U(log dt_range[0], log dt_range[1]) (fp32; the default is
+    Mamba's initialisation range, whose fastest channels decay beyond the
+    factorised chunk range in most chunks), beta, S0 and cu_seqlens as
+    make_inputs."""
     g = torch.Generator(device=device).manual_seed(seed)
     N = len(seqlens) if seqlens is not None else B
     if seqlens is not None and (B != 1 or T != sum(seqlens)):
@@ -171,7 +173,8 @@ def make_layer_inputs(B: int, T: int, H: int, dk: int, dv: int, *, dtype=torch.b
     v = _normal((B, T, H, dv), g, device)
     f = _normal((B, T, H, dk), g, device)
     A_log = torch.log(1.0 + 15.0 * torch.rand((H,), generator=g, device=device))
-    dt = torch.exp(math.log(1e-3) + (math.log(1e-1) - math.log(1e-3)) * torch.rand((H, dk), generator=g, device=device))
+    lo, hi = math.log(dt_range[0]), math.log(dt_range[1])
+    dt = torch.exp(lo + (hi - lo) * torch.rand((H, dk), generator=g, device=device))
     dt_bias = dt + torch.log(-torch.expm1(-dt))
     beta = torch.sigmoid(_normal((B, T, H), g, device))
     S0 = 0.1 * _normal((N, H, dk, dv), g, device)

@@ -52,7 +52,7 @@
 extern "C" {
 #endif
 
-#define KDA_ABI_VERSION 4
+#define KDA_ABI_VERSION 5
 
 typedef enum {
   KDA_OK = 0,
@@ -181,6 +181,42 @@ kda_status kda_chunk_fwd_gated(const kda_shape* shape, const void* q, const void
                                const void* log_alpha, const void* beta, const float* S0, const int32_t* cu_seqlens,
                                const void* out_gate, const float* norm_weight, float eps, void* o, float* S_T,
                                void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * kda_chunk_fwd_layer -- the operator as the Kimi Linear layer uses it, with
+ * its producer steps done inside the prefill kernel (the "Kimi Linear"
+ * summary, section "Configuração do modelo Kimi Linear": q and k are
+ * L2-normalised for the stability of the transition's eigenvalues; the
+ * channel-wise decay gate comes from a low-rank projection through a decay
+ * function like GDN's and Mamba's) and, optionally, its consumer step (the
+ * per-head RMSNorm and output gate of kda_chunk_fwd_gated).  Equivalent to
+ *
+ *     kda_chunk_fwd(q / |q|, k / |k|, v, log_alpha, beta, ...)   with
+ *     |x| = sqrt(sum_c x[c]^2 + KDA_QK_NORM_EPS) per (token, head) row and
+ *     log_alpha[t][h][c] = -exp(A_log[h]) * softplus(gate_f[t][h][c] + dt_bias[h][c])
+ *
+ * followed by the output epilogue when out_gate is not NULL, without the
+ * normalised q, k or log_alpha ever reaching HBM.
+ *
+ *   q, k      raw (not normalised) [B, T, H, dk] bf16.
+ *   gate_f    the decay gate's projection output, [B, T, H, dk] bf16.
+ *   A_log     [H] fp32 (the per-head rate is exp(A_log)); 4-byte aligned.
+ *   dt_bias   [H, dk] fp32; 16-byte aligned.
+ *   out_gate, norm_weight, eps   as kda_chunk_fwd_gated, or out_gate and
+ *             norm_weight both NULL for no epilogue (one NULL: KDA_ERR_NULL).
+ * Everything else as kda_chunk_fwd.  Only the tensor-core path (bf16 io and
+ * gates, dk = dv = 128, no KDA_FLAG_PATH_RECURRENT) runs the producer steps:
+ * other shapes return KDA_ERR_UNSUPPORTED.  softplus and exp are evaluated in
+ * fp32 with the hardware 2^x and log2 approximations, and log alpha enters
+ * the chunk's cumulative sum with 16 significant bits (relative error below
+ * 2^-16; the bf16 log_alpha of kda_chunk_fwd carries 8).
+ */
+#define KDA_QK_NORM_EPS 1e-6f
+kda_status kda_chunk_fwd_layer(const kda_shape* shape, const void* q, const void* k, const void* v,
+                               const void* gate_f, const float* A_log, const float* dt_bias, const void* beta,
+                               const float* S0, const int32_t* cu_seqlens, const void* out_gate,
+                               const float* norm_weight, float eps, void* o, float* S_T, void* workspace,
+                               size_t workspace_bytes, void* stream);
 
 /*
  * kda_chunk_fwd_noalloc -- kda_chunk_fwd for callers that cannot allocate.

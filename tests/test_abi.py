@@ -30,7 +30,7 @@ def test_library_loads_and_exports_every_declared_symbol():
     lib = kda.load_library()
     for name in declared_functions():
         assert hasattr(lib, name), name
-    assert kda.kda_abi_version() == 4
+    assert kda.kda_abi_version() == 5
 
 
 def test_status_strings():
@@ -181,6 +181,31 @@ def test_gated_prefill_host_validation():
     for shape in (tc_shape(io_dtype=0), tc_shape(dk=64, dv=64), tc_shape(flags=kda.KDA_FLAG_PATH_RECURRENT),
                   tc_shape(B=2, T=200), tc_shape(flags=kda.KDA_FLAG_GATE_SEPARATE)):
         assert call_fwd_gated(shape) in (-6, -7)
+
+
+def call_fwd_layer(shape, A=FAKE, bias=FAKE, gate=None, weight=None, eps=1e-5):
+    lib = kda.load_library()
+    vp = lambda x: None if x is None else ctypes.c_void_p(x)
+    f = vp(FAKE)
+    return lib.kda_chunk_fwd_layer(ctypes.byref(shape), f, f, f, f, vp(A), vp(bias), f, None, None, vp(gate),
+                                   vp(weight), ctypes.c_float(eps), f, None, None, 0, None)
+
+
+def test_layer_prefill_host_validation():
+    assert call_fwd_layer(tc_shape(), A=None) == -1
+    assert call_fwd_layer(tc_shape(), bias=None) == -1
+    assert call_fwd_layer(tc_shape(), A=FAKE + 2) == -4
+    assert call_fwd_layer(tc_shape(), bias=FAKE + 4) == -4
+    assert call_fwd_layer(tc_shape(), gate=FAKE) == -1
+    assert call_fwd_layer(tc_shape(), weight=FAKE) == -1
+    assert call_fwd_layer(tc_shape(), gate=FAKE, weight=FAKE, eps=-1.0) == -10
+    assert call_fwd_layer(tc_shape(), gate=FAKE + 2, weight=FAKE) == -4
+    # the producer steps run in the tensor-core kernel only
+    for shape in (tc_shape(io_dtype=0), tc_shape(gate_dtype=0), tc_shape(dk=64, dv=64),
+                  tc_shape(flags=kda.KDA_FLAG_PATH_RECURRENT)):
+        assert call_fwd_layer(shape) == -5
+    assert call_fwd_layer(tc_shape(B=2, T=200)) in (-6, -7)
+    assert call_fwd_layer(tc_shape(B=2, T=200), gate=FAKE, weight=FAKE) in (-6, -7)
 
 
 def test_python_binding_refuses_cpu_tensors():
