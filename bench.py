@@ -307,13 +307,26 @@ def cpu_model() -> str:
     return "unknown"
 
 
+# The layer legs' decay-gate parameters: Mamba's A range with step sizes
+# dt in [1e-3, 1e-2], so that chunk decays stay in the factorised range as in
+# the plain workloads (the default dt range up to 0.1 sends some chunks of
+# the fastest channels to the exact path).
+LAYER_DT_RANGE = (1e-3, 1e-2)
+
+
 def prefill_leg(kda, gen, wname, steps, warmup, world, rank, local, stream, peaks, peak_src, counters,
-                gated=False):
+                gated=False, layer=False):
     """Times kda_chunk_fwd (kda_chunk_fwd_gated with ``gated``: the output
-    RMSNorm and sigmoid gate, placed by the library) on one workload; returns
-    its JSON object."""
+    RMSNorm and sigmoid gate, placed by the library; kda_chunk_fwd_layer with
+    ``layer``: raw q, k and the gate projection in, L2 norm and decay gate in
+    the kernel, plus the output epilogue) on one workload; returns its JSON
+    object."""
     w = gen.workload(wname)
-    x = gen.workload_inputs(w, device="cuda", seed_offset=rank)
+    if layer:
+        x = gen.make_layer_inputs(w.B, w.T, w.H, w.dk, w.dv, seqlens=w.seqlens, seed=w.seed + rank, device="cuda",
+                                  dt_range=LAYER_DT_RANGE)
+    else:
+        x = gen.workload_inputs(w, device="cuda", seed_offset=rank)
     cu = x["cu_seqlens"]
     n_seqs = 0 if cu is None else cu.numel() - 1
     N = w.B if cu is None else n_seqs
@@ -321,7 +334,13 @@ def prefill_leg(kda, gen, wname, steps, warmup, world, rank, local, stream, peak
     ws = torch.empty(max(kda.kda_chunk_fwd_workspace_size(shape), 1), dtype=torch.uint8, device="cuda")
     o = torch.empty_like(x["v"])
     S_T = torch.empty_like(x["S0"])
-    if gated:
+    if layer:
+        gate, nw = gen.output_gate_inputs(x["v"].shape, seed=w.seed + 100 + rank, device="cuda")
+
+        def fn():
+            kda.kda_chunk_fwd_layer(x["q"], x["k"], x["v"], x["f"], x["A_log"], x["dt_bias"], x["beta"], x["S0"], cu,
+                                    out_gate=gate, norm_weight=nw, eps=1e-5, o=o, S_T=S_T, workspace=ws)
+    elif gated:
         gate, nw = gen.output_gate_inputs(x["v"].shape, seed=w.seed + 100 + rank, device="cuda")
 
         def fn():
@@ -332,7 +351,7 @@ def prefill_leg(kda, gen, wname, steps, warmup, world, rank, local, stream, peak
             kda.kda_chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["S0"], cu, o=o, S_T=S_T,
                               workspace=ws)
 
-    label = wname + (" gated" if gated else "")
+    label = wname + (" layer" if layer else " gated" if gated else "")
     progress(f"{label}: timing {steps} calls")
     with ClockSampler(local) as clk:
         t = timed(fn, steps, warmup, world, stream)
@@ -342,19 +361,22 @@ def prefill_leg(kda, gen, wname, steps, warmup, world, rank, local, stream, peak
     tokens = w.B * w.T
     ms = t / steps * 1e3
     nbytes = prefill_bytes(tokens, 1, w.H, w.dk) - 2 * tokens * w.H * w.dk * w.dk * 4 + 2 * N * w.H * w.dk * w.dk * 4
-    if gated:
+    if gated or layer:
         nbytes += tokens * w.H * w.dv * 2 + w.dv * 4  # the gate read, the norm weight
     flops = prefill_flops(tokens, 1, w.H, w.dk)
     gbs = nbytes / (ms / 1e3) / 1e9
     peak = float(peaks["hbm_gbs"])
-    c = counters.get(wname + ("_gated" if gated else ""), {})
+    c = counters.get(wname + ("_layer" if layer else "_gated" if gated else ""), {})
     traffic = c.get("dram_bytes")
     progress(f"{label}: {ms:.3f} ms/call, {gbs:.0f} GB/s")
     out = {
         "value": tokens * world * steps / t, "unit": "tokens/s", "ms_per_step": ms, "steps": steps,
         "config": {"workload": f"{wname} {w.B}x{w.T} tokens H{w.H} dk=dv={w.dk} C64, bf16 q/k/v/gates, fp32 state"
                                + (", then per-head RMSNorm + sigmoid output gate (bf16 gate; fused into the prefill kernel "
-                                  "where its transform CTAs bound the call, else a separate pass over o)" if gated else ""),
+                                  "where its transform CTAs bound the call, else a separate pass over o)" if gated else "")
+                               + (": raw q, k and decay-gate projection f in (L2 norm of q, k and log alpha = "
+                                  "-exp(A_log) softplus(f + dt_bias) computed in the kernel; A ~ U(1,16), "
+                                  "dt ~ logU(1e-3, 1e-2)), per-head RMSNorm + sigmoid output gate out" if layer else ""),
                    "sequences": N, "tokens": tokens, "H": w.H,
                    "l2": f"inputs larger than L2 (no flush): {tokens * w.H * w.dk * 8 / 1e6:.0f} MB read per call"},
         "roofline": {"kernel": "kda_prefill_kernel (one cooperative launch per call)", "bound": "hbm",
@@ -366,7 +388,7 @@ def prefill_leg(kda, gen, wname, steps, warmup, world, rank, local, stream, peak
         "clocks": clk.summary(),
     }
     del x, ws, o, S_T
-    if gated:
+    if gated or layer:
         del gate, nw
     torch.cuda.empty_cache()
     return out
@@ -436,6 +458,12 @@ def run_ours(args):
     lgt = prefill_leg(kda, gen, "long", long_steps, args.warmup, world, rank, local, stream, peaks, peak_src,
                       counters, gated=True)
     launches += 2 * long_steps  # the prefill kernel and the separate epilogue pass
+    ply = prefill_leg(kda, gen, "prefill", args.steps, args.warmup, world, rank, local, stream, peaks, peak_src,
+                      counters, layer=True)
+    launches += args.steps
+    lly = prefill_leg(kda, gen, "long", long_steps, args.warmup, world, rank, local, stream, peaks, peak_src,
+                      counters, layer=True)
+    launches += 2 * long_steps
 
     # ---------------- decode
     progress("decode: setup")
@@ -488,6 +516,8 @@ def run_ours(args):
             "prefill_gated": gtd,
             "varlen_gated": vgt,
             "long_gated": lgt,
+            "prefill_layer": ply,
+            "long_layer": lly,
             "decode": {"value": world * dec_steps / t_dec, "unit": "steps/s", "ms_per_step": dec_ms,
                        "steps": dec_steps,
                        "config": {"workload": "decode 256 seqs x H32 dk=dv=128, fp32 state 537 MB in place, "
@@ -515,7 +545,7 @@ def run_profile(args):
     torch.cuda.set_device(0)
     kda.load_library()
     stream = torch.cuda.current_stream()
-    w = gen.workload("prefill" if args.profile.startswith("gated") else args.profile)
+    w = gen.workload("prefill" if args.profile.startswith("gated") or args.profile == "layer" else args.profile)
     if args.profile == "decode":
         S = gen.decode_state(w.B, w.H, w.dk, w.dv, device="cuda", seed=w.seed)
         xs = gen.decode_step_inputs(w.B, w.H, w.dk, w.dv, 0, device="cuda", seed=w.seed)
@@ -524,19 +554,25 @@ def run_profile(args):
         def fn():
             kda.kda_decode_step(xs["q"], xs["k"], xs["v"], xs["log_alpha"], xs["beta"], S, o=od)
     else:
-        x = gen.workload_inputs(w, device="cuda")
+        if args.profile == "layer":
+            x = gen.make_layer_inputs(w.B, w.T, w.H, w.dk, w.dv, seed=w.seed, device="cuda", dt_range=LAYER_DT_RANGE)
+        else:
+            x = gen.workload_inputs(w, device="cuda")
         n_seqs = 0 if x["cu_seqlens"] is None else x["cu_seqlens"].numel() - 1
         shape = kda.make_shape(w.B, w.T, w.H, w.dk, w.dv, 64, n_seqs, kda.KDA_BF16, kda.KDA_BF16)
         ws = torch.empty(max(kda.kda_chunk_fwd_workspace_size(shape), 1), dtype=torch.uint8, device="cuda")
         o = torch.empty_like(x["v"])
         S_T = torch.empty_like(x["S0"])
 
-        if args.profile.startswith("gated"):
+        if args.profile.startswith("gated") or args.profile == "layer":
             gate, nw = gen.output_gate_inputs(x["v"].shape, seed=w.seed + 100, device="cuda")
             mode = "separate" if args.profile == "gated_separate" else "fused"
 
         def fn():
-            if args.profile.startswith("gated"):
+            if args.profile == "layer":
+                kda.kda_chunk_fwd_layer(x["q"], x["k"], x["v"], x["f"], x["A_log"], x["dt_bias"], x["beta"], x["S0"],
+                                        out_gate=gate, norm_weight=nw, eps=1e-5, o=o, S_T=S_T, workspace=ws)
+            elif args.profile.startswith("gated"):
                 kda.kda_chunk_fwd_gated(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], gate, nw, x["S0"],
                                         x["cu_seqlens"], eps=1e-5, o=o, S_T=S_T, workspace=ws, gate_mode=mode)
             else:
@@ -562,7 +598,7 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=1000)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", choices=("prefill", "varlen", "long", "decode", "gated", "gated_separate"),
+    ap.add_argument("--profile", choices=("prefill", "varlen", "long", "decode", "gated", "gated_separate", "layer"),
                     default=None,
                     help="time one workload's entry point alone (for ncu); prints no JSON line")
     args = ap.parse_args()
