@@ -72,24 +72,29 @@ def _lengths(q, cu_seqlens):
     return [c[i + 1] - c[i] for i in range(len(c) - 1)]
 
 
-def local_inputs(plan: ShardPlan, q, k, v, log_alpha, beta, S0=None, cu_seqlens=None):
+def local_inputs(plan: ShardPlan, q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, token_extras=(),
+                 head_extras=()):
     """This rank's slice of the inputs, in the library's layouts.
 
-    Returns (q, k, v, log_alpha, beta, S0, cu_seqlens) for the shard; for a
-    sequence shard of a packed batch, cu_seqlens is rebased to start at 0."""
+    Returns (q, k, v, log_alpha, beta, S0, cu_seqlens, *token_extras,
+    *head_extras) for the shard; for a sequence shard of a packed batch,
+    cu_seqlens is rebased to start at 0.  ``token_extras`` are laid out like
+    q ([B, T, H, ...]) and sliced with it; ``head_extras`` have the head
+    axis first ([H, ...]) and are sliced only by a head shard."""
     if plan.kind == "seq":
         if cu_seqlens is None:
             sl = slice(plan.n0, plan.n1)
-            xs = [t[sl] for t in (q, k, v, log_alpha, beta)]
-            return (*xs, None if S0 is None else S0[sl], None)
+            xs = [t[sl] for t in (q, k, v, log_alpha, beta, *token_extras)]
+            return (*xs[:5], None if S0 is None else S0[sl], None, *xs[5:], *head_extras)
         c = cu_seqlens
         a, e = int(c[plan.n0]), int(c[plan.n1])
-        xs = [t[:, a:e] for t in (q, k, v, log_alpha, beta)]
+        xs = [t[:, a:e] for t in (q, k, v, log_alpha, beta, *token_extras)]
         cu = (c[plan.n0:plan.n1 + 1] - c[plan.n0]).contiguous()
-        return (*xs, None if S0 is None else S0[plan.n0:plan.n1], cu)
+        return (*xs[:5], None if S0 is None else S0[plan.n0:plan.n1], cu, *xs[5:], *head_extras)
     hs = slice(plan.h0, plan.h1)
-    xs = [t[:, :, hs].contiguous() for t in (q, k, v, log_alpha, beta)]
-    return (*xs, None if S0 is None else S0[:, hs].contiguous(), cu_seqlens)
+    xs = [t[:, :, hs].contiguous() for t in (q, k, v, log_alpha, beta, *token_extras)]
+    hx = [t[hs].contiguous() for t in head_extras]
+    return (*xs[:5], None if S0 is None else S0[:, hs].contiguous(), cu_seqlens, *xs[5:], *hx)
 
 
 def _gather_padded(t, group, dist):
@@ -108,14 +113,15 @@ def _gather_padded(t, group, dist):
 
 
 def kda_chunk_fwd_sharded(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, *, group=None, fwd=None,
-                          gather: bool = True):
+                          gather: bool = True, token_extras=(), head_extras=()):
     """Prefill of a batch split across the ranks of ``group``.
 
     Every rank passes the same full inputs (or at least the same shapes and
-    cu_seqlens; only its own shard is read).  ``fwd`` computes one shard and
-    defaults to the library's kda_chunk_fwd.  With ``gather`` every rank
-    returns the full (o, S_T); otherwise its own shard, its plan, and no
-    collective is issued.
+    cu_seqlens; only its own shard is read).  ``fwd`` computes one shard,
+    called as fwd(q, k, v, log_alpha, beta, S0, cu_seqlens, *token_extras,
+    *head_extras) on the shard's slices (see local_inputs), and defaults to
+    the library's kda_chunk_fwd.  With ``gather`` every rank returns the full
+    (o, S_T); otherwise its own shard, its plan, and no collective is issued.
     """
     import torch
     import torch.distributed as dist
@@ -126,13 +132,14 @@ def kda_chunk_fwd_sharded(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, *,
     H = q.shape[2]
     plans = plan_shards(_lengths(q, cu_seqlens), H, world)
     plan = plans[rank]
-    lq, lk, lv, la, lb, ls0, lcu = local_inputs(plan, q, k, v, log_alpha, beta, S0, cu_seqlens)
+    loc = local_inputs(plan, q, k, v, log_alpha, beta, S0, cu_seqlens, token_extras, head_extras)
+    lq, lv = loc[0], loc[2]
     empty = (plan.n1 - plan.n0) == 0 or (plan.h1 - plan.h0) == 0
     if empty:
         o_loc = lv.new_zeros(lv.shape)
-        S_loc = q.new_zeros((plan.n1 - plan.n0, plan.h1 - plan.h0, q.shape[3], v.shape[3]), dtype=torch.float32)
+        S_loc = lq.new_zeros((plan.n1 - plan.n0, plan.h1 - plan.h0, q.shape[3], v.shape[3]), dtype=torch.float32)
     else:
-        o_loc, S_loc = fwd(lq, lk, lv, la, lb, ls0, lcu)
+        o_loc, S_loc = fwd(*loc)
     if not gather or world == 1:
         return o_loc, S_loc, plan
     # rows of o along the sharded axis first, so that shards concatenate
@@ -151,3 +158,27 @@ def kda_chunk_fwd_sharded(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, *,
     o = torch.cat(o_parts, 0).permute(1, 2, 0, 3).contiguous()
     S_T = torch.cat(S_parts, 0).permute(1, 0, 2, 3).contiguous()
     return o, S_T, plan
+
+
+def kda_chunk_fwd_layer_sharded(q, k, v, gate_f, A_log, dt_bias, beta, S0=None, cu_seqlens=None, *, out_gate=None,
+                                norm_weight=None, eps: float = 1e-5, group=None, fwd=None, gather: bool = True):
+    """kda_chunk_fwd_layer (raw q, k and the decay gate's projection in; the
+    optional output epilogue) split across the ranks of ``group`` as
+    kda_chunk_fwd_sharded splits kda_chunk_fwd: gate_f and out_gate are
+    sliced like q, A_log and dt_bias by head.  ``fwd`` (default: the
+    library's kda_chunk_fwd_layer) is called as fwd(q, k, v, gate_f, beta,
+    S0, cu_seqlens, out_gate, A_log, dt_bias, norm_weight=..., eps=...)."""
+    if fwd is None:
+        from . import kda_chunk_fwd_layer
+
+        def fwd(lq, lk, lv, lf, lb, ls0, lcu, lgate, lA, lbias, norm_weight=None, eps=1e-5):
+            return kda_chunk_fwd_layer(lq, lk, lv, lf, lA, lbias, lb, ls0, lcu, out_gate=lgate,
+                                       norm_weight=norm_weight, eps=eps)
+    tok = (out_gate,) if out_gate is not None else ()
+
+    def shard_fwd(lq, lk, lv, lf, lb, ls0, lcu, *rest):
+        lgate = rest[0] if out_gate is not None else None
+        lA, lbias = rest[-2], rest[-1]
+        return fwd(lq, lk, lv, lf, lb, ls0, lcu, lgate, lA, lbias, norm_weight=norm_weight, eps=eps)
+    return kda_chunk_fwd_sharded(q, k, v, gate_f, beta, S0, cu_seqlens, group=group, fwd=shard_fwd, gather=gather,
+                                 token_extras=tok, head_extras=(A_log, dt_bias))

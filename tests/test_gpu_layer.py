@@ -120,3 +120,19 @@ def test_layer_prefill_workload_sampled():
         sub["S0"] = x["S0"][b:b + 1, h:h + 1].cpu()
         sub["cu_seqlens"] = None
         _check(sub, o[b:b + 1, :, h:h + 1], S[b:b + 1, h:h + 1], gate[b:b + 1, :, h:h + 1].cpu(), w.cpu(), 1e-5)
+
+
+def test_layer_sharded_single_rank_is_the_plain_call():
+    """kda_chunk_fwd_layer_sharded without a process group runs the library's
+    call on the whole batch (the multi-rank split is tested on CPU)."""
+    from gated_delta_rule_110_b200.shard import kda_chunk_fwd_layer_sharded
+    lens = [70, 130, 64]
+    x = {k: (v.cuda() if isinstance(v, torch.Tensor) else v)
+         for k, v in gen.make_layer_inputs(1, sum(lens), 2, 128, 128, seqlens=lens, seed=70).items()}
+    gate, w = gen.output_gate_inputs(x["v"].shape, seed=71, device="cuda")
+    o1, S1, _ = kda_chunk_fwd_layer_sharded(x["q"], x["k"], x["v"], x["f"], x["A_log"], x["dt_bias"], x["beta"],
+                                            x["S0"], x["cu_seqlens"], out_gate=gate, norm_weight=w)
+    o2, S2 = kda.kda_chunk_fwd_layer(x["q"], x["k"], x["v"], x["f"], x["A_log"], x["dt_bias"], x["beta"], x["S0"],
+                                     x["cu_seqlens"], out_gate=gate, norm_weight=w)
+    assert kda.kda_check_device_error() == 0
+    assert torch.equal(o1, o2) and torch.equal(S1, S2)

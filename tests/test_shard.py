@@ -103,3 +103,52 @@ def test_two_gloo_ranks_gather_the_unsharded_result(tmp_path, name, kind):
         assert got["kind"] == kind
         assert torch.equal(got["o"], o_ref), f"rank {r}: o differs"
         assert torch.equal(got["S"], S_ref), f"rank {r}: S_T differs"
+
+
+# ---------------------------------------------------------------- the layer path
+def _oracle_layer_fwd(q, k, v, f, beta, S0, cu, gate, A_log, dt_bias, norm_weight=None, eps=1e-5):
+    import oracle
+    o, S = oracle.forward_layer(q, k, v, f, A_log, dt_bias, beta, S0, cu_seqlens=None if cu is None else cu.numpy(),
+                                out_gate=gate, norm_weight=norm_weight, eps=eps)
+    return torch.from_numpy(o), torch.from_numpy(S)
+
+
+def _layer_case(name):
+    if name == "packed":
+        lens = [70, 0, 130, 1, 64, 200]
+        x = gen.make_layer_inputs(1, sum(lens), 2, 32, 32, dtype=torch.float32, seqlens=lens, seed=71)
+    else:
+        x = gen.make_layer_inputs(1, 150, 4, 32, 32, dtype=torch.float32, seqlens=[150], seed=72)
+    gate, w = gen.output_gate_inputs(x["v"].shape, dtype=torch.float32, seed=73)
+    return x, gate, w
+
+
+def _layer_rank_main(rank, world, port, name, out_dir):
+    import torch.distributed as dist
+    from gated_delta_rule_110_b200.shard import kda_chunk_fwd_layer_sharded
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world)
+    try:
+        x, gate, w = _layer_case(name)
+        o, S, plan = kda_chunk_fwd_layer_sharded(x["q"], x["k"], x["v"], x["f"], x["A_log"], x["dt_bias"], x["beta"],
+                                                 x["S0"], x["cu_seqlens"], out_gate=gate, norm_weight=w, eps=1e-5,
+                                                 fwd=_oracle_layer_fwd)
+        torch.save({"o": o, "S": S, "kind": plan.kind}, os.path.join(out_dir, f"r{rank}.pt"))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("name,kind", [("packed", "seq"), ("heads", "head")])
+def test_two_gloo_ranks_layer_path(tmp_path, name, kind):
+    """The layer path's extra inputs shard with the rest: the gate projection
+    and the output gate with the tokens, A_log and dt_bias with the heads."""
+    world = 2
+    mp.start_processes(_layer_rank_main, args=(world, _free_port(), name, str(tmp_path)), nprocs=world,
+                       start_method="spawn", join=True)
+    x, gate, w = _layer_case(name)
+    o_ref, S_ref = _oracle_layer_fwd(x["q"], x["k"], x["v"], x["f"], x["beta"], x["S0"], x["cu_seqlens"], gate,
+                                     x["A_log"], x["dt_bias"], norm_weight=w, eps=1e-5)
+    for r in range(world):
+        got = torch.load(tmp_path / f"r{r}.pt")
+        assert got["kind"] == kind
+        assert torch.equal(got["o"], o_ref), f"rank {r}: o differs"
+        assert torch.equal(got["S"], S_ref), f"rank {r}: S_T differs"
