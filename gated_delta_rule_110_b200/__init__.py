@@ -14,6 +14,8 @@ Entry points (same names as the C ABI):
   (sequence, head), ``S`` updated in place -> ``o``
 * ``kda_chunk_fwd_layer(q, k, v, gate_f, A_log, dt_bias, beta, ...)`` raw q, k and
   the decay gate's projection in (L2 norm and gate computed in the kernel) -> ``(o, S_T)``
+* ``kda_decode_step_layer(q, k, v, gate_f, A_log, dt_bias, beta, state, ...)`` one
+  decode step with the layer's producer steps (and optional output epilogue)
 * ``kda_chunk_fwd_gated(q, k, v, log_alpha, beta, out_gate, norm_weight, ...)``
   prefill with the per-head RMSNorm and sigmoid output gate fused -> ``(o', S_T)``
 * ``kda_chunk_fwd_slots(q, k, v, log_alpha, beta, state_pool, state_slots,
@@ -50,7 +52,7 @@ EXPORTED_SYMBOLS = (
     "kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_chunk_fwd_gated", "kda_chunk_fwd_layer",
     "kda_chunk_fwd_noalloc",
     "kda_chunk_fwd_slots",
-    "kda_decode_step", "kda_decode_step_slots", "kda_check_device_error", "kda_status_string",
+    "kda_decode_step", "kda_decode_step_slots", "kda_decode_step_layer", "kda_check_device_error", "kda_status_string",
     "kda_abi_version",
 )
 
@@ -99,6 +101,9 @@ def load_library(build_if_missing: bool = True):
     lib.kda_chunk_fwd_layer.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp, vp,
                                         ctypes.c_size_t, vp]
     lib.kda_chunk_fwd_layer.restype = ctypes.c_int
+    lib.kda_decode_step_layer.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_int32, vp, vp,
+                                          ctypes.c_float, vp, vp]
+    lib.kda_decode_step_layer.restype = ctypes.c_int
     lib.kda_chunk_fwd_noalloc.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.kda_chunk_fwd_noalloc.restype = ctypes.c_int
     lib.kda_chunk_fwd_slots.argtypes = [sp, vp, vp, vp, vp, vp, vp, ctypes.c_int32, vp, vp, vp, vp, vp,
@@ -249,7 +254,7 @@ def kda_chunk_fwd_gated(q, k, v, log_alpha, beta, out_gate, norm_weight, S0=None
 def kda_chunk_fwd_layer(q, k, v, gate_f, A_log, dt_bias, beta, S0=None, cu_seqlens=None, *, out_gate=None,
                         norm_weight=None, eps: float = 1e-5, chunk: int = 64, o=None, S_T=None, workspace=None,
                         stream=None, validate: bool = False, output_final_state: bool = True,
-                        gate_mode: str = "auto", state_ctas: int = 0, grid_ctas: int = 0):
+                        recurrent: bool = False, gate_mode: str = "auto", state_ctas: int = 0, grid_ctas: int = 0):
     """The operator with the Kimi Linear layer's producer steps fused (raw q,
     k are L2-normalised, log alpha = -exp(A_log) * softplus(gate_f + dt_bias))
     and, with ``out_gate`` / ``norm_weight``, its output epilogue
@@ -270,7 +275,7 @@ def kda_chunk_fwd_layer(q, k, v, gate_f, A_log, dt_bias, beta, S0=None, cu_seqle
             raise ValueError("norm_weight must be a float32 tensor of dv values")
     if gate_mode not in _GATE_MODES:
         raise ValueError(f"gate_mode must be one of {sorted(_GATE_MODES)}")
-    shape = _shape_of(q, v, gate_f, cu_seqlens, chunk, validate, False, state_ctas, grid_ctas)
+    shape = _shape_of(q, v, gate_f, cu_seqlens, chunk, validate, recurrent, state_ctas, grid_ctas)
     shape.flags |= _GATE_MODES[gate_mode]
     N = shape.B if cu_seqlens is None else shape.n_seqs
     if o is None:
@@ -288,6 +293,40 @@ def kda_chunk_fwd_layer(q, k, v, gate_f, A_log, dt_bias, beta, S0=None, cu_seqle
     if rc != KDA_OK:
         raise KdaError(rc, "kda_chunk_fwd_layer")
     return o, S_T
+
+
+def kda_decode_step_layer(q, k, v, gate_f, A_log, dt_bias, beta, state, *, state_slots=None, out_gate=None,
+                          norm_weight=None, eps: float = 1e-5, o=None, stream=None):
+    """One decode step with the layer's producer steps (raw q, k; decay gate
+    from gate_f, A_log, dt_bias) and the optional output epilogue; ``state``
+    is updated in place (dense rows, or pool slots with ``state_slots``).
+    Inputs [N, H, d] (one token per sequence) or [N, 1, H, d]; returns o."""
+    import torch
+    _need_cuda(q, k, v, gate_f, A_log, dt_bias, beta, state, state_slots, out_gate, norm_weight, o)
+    if q.dim() == 3:
+        q, k, v, gate_f = (t.unsqueeze(1) for t in (q, k, v, gate_f))
+        beta = beta.unsqueeze(1)
+        if out_gate is not None:
+            out_gate = out_gate.unsqueeze(1)
+    N, _, H, dk = q.shape
+    if (out_gate is None) != (norm_weight is None):
+        raise ValueError("out_gate and norm_weight go together")
+    if A_log.dtype != torch.float32 or dt_bias.dtype != torch.float32:
+        raise ValueError("A_log and dt_bias must be float32")
+    shape = _shape_of(q, v, gate_f, None, 64, False)
+    if o is None:
+        o = torch.empty((N, H, v.shape[-1]), dtype=v.dtype, device=v.device)
+    num_slots = 0
+    if state_slots is not None:
+        _check_slots(state, state_slots, N)
+        num_slots = state.shape[0]
+    rc = load_library().kda_decode_step_layer(
+        ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(gate_f), _ptr(A_log), _ptr(dt_bias), _ptr(beta),
+        _ptr(state), _ptr(state_slots), num_slots, _ptr(out_gate), _ptr(norm_weight), float(eps), _ptr(o),
+        _stream(stream))
+    if rc != KDA_OK:
+        raise KdaError(rc, "kda_decode_step_layer")
+    return o
 
 
 def kda_chunk_fwd_noalloc(q, k, v, log_alpha, beta, S0, cu_seqlens, o, S_T, *, chunk: int = 64, stream=None,

@@ -66,46 +66,54 @@ kda_status launch_status() {
 template <int DK, int DV, typename TIO, typename TG>
 kda_status launch_recurrent_fwd(const kda_shape& s, int64_t N, const void* q, const void* k, const void* v,
                                 const void* la, const void* beta, const kda::StateIO& io, const int32_t* cu,
-                                void* o, cudaStream_t st) {
+                                void* o, cudaStream_t st, const kda::RecProducer& pr, const kda::RecConsumer& cs) {
   dim3 grid(s.H, static_cast<unsigned>(N));
-  kda::kda_recurrent_fwd_kernel<DK, DV, TIO, TG><<<grid, kda::kRecThreads, 0, st>>>(
-      s.H, s.T, cu, static_cast<const TIO*>(q), static_cast<const TIO*>(k), static_cast<const TIO*>(v),
-      static_cast<const TG*>(la), static_cast<const TG*>(beta), io, static_cast<TIO*>(o));
+  auto* kern = pr.A_log ? kda::kda_recurrent_fwd_kernel<DK, DV, TIO, TG, true>
+                        : kda::kda_recurrent_fwd_kernel<DK, DV, TIO, TG, false>;
+  kern<<<grid, kda::kRecThreads, 0, st>>>(s.H, s.T, cu, static_cast<const TIO*>(q), static_cast<const TIO*>(k),
+                                          static_cast<const TIO*>(v), static_cast<const TG*>(la),
+                                          static_cast<const TG*>(beta), io, static_cast<TIO*>(o), pr, cs);
   return launch_status();
 }
 
 template <typename TIO, typename TG>
 kda_status dispatch_recurrent_fwd(const kda_shape& s, int64_t N, const void* q, const void* k, const void* v,
                                   const void* la, const void* beta, const kda::StateIO& io, const int32_t* cu,
-                                  void* o, cudaStream_t st) {
+                                  void* o, cudaStream_t st, const kda::RecProducer& pr,
+                                  const kda::RecConsumer& cs) {
   if (s.dk == 128 && s.dv == 128)
-    return launch_recurrent_fwd<128, 128, TIO, TG>(s, N, q, k, v, la, beta, io, cu, o, st);
+    return launch_recurrent_fwd<128, 128, TIO, TG>(s, N, q, k, v, la, beta, io, cu, o, st, pr, cs);
   if (s.dk == 64 && s.dv == 64)
-    return launch_recurrent_fwd<64, 64, TIO, TG>(s, N, q, k, v, la, beta, io, cu, o, st);
+    return launch_recurrent_fwd<64, 64, TIO, TG>(s, N, q, k, v, la, beta, io, cu, o, st, pr, cs);
   if (s.dk == 128 && s.dv == 64)
-    return launch_recurrent_fwd<128, 64, TIO, TG>(s, N, q, k, v, la, beta, io, cu, o, st);
-  return launch_recurrent_fwd<64, 128, TIO, TG>(s, N, q, k, v, la, beta, io, cu, o, st);
+    return launch_recurrent_fwd<128, 64, TIO, TG>(s, N, q, k, v, la, beta, io, cu, o, st, pr, cs);
+  return launch_recurrent_fwd<64, 128, TIO, TG>(s, N, q, k, v, la, beta, io, cu, o, st, pr, cs);
 }
 
 template <int DK, int DV, typename TIO, typename TG>
 kda_status launch_decode(const kda_shape& s, const void* q, const void* k, const void* v, const void* la,
                          const void* beta, float* S, const int32_t* slots, int num_slots, void* o,
-                         cudaStream_t st) {
+                         cudaStream_t st, const kda::RecProducer& pr, const kda::RecConsumer& cs) {
   const unsigned blocks = static_cast<unsigned>(s.B) * static_cast<unsigned>(s.H);
-  kda::kda_decode_kernel<DK, DV, TIO, TG><<<blocks, kda::kRecThreads, 0, st>>>(
-      s.H, static_cast<const TIO*>(q), static_cast<const TIO*>(k), static_cast<const TIO*>(v),
-      static_cast<const TG*>(la), static_cast<const TG*>(beta), S, static_cast<TIO*>(o), slots, num_slots);
+  auto* kern = pr.A_log ? kda::kda_decode_kernel<DK, DV, TIO, TG, true> : kda::kda_decode_kernel<DK, DV, TIO, TG, false>;
+  kern<<<blocks, kda::kRecThreads, 0, st>>>(s.H, static_cast<const TIO*>(q), static_cast<const TIO*>(k),
+                                            static_cast<const TIO*>(v), static_cast<const TG*>(la),
+                                            static_cast<const TG*>(beta), S, static_cast<TIO*>(o), slots, num_slots,
+                                            pr, cs);
   return launch_status();
 }
 
 template <typename TIO, typename TG>
 kda_status dispatch_decode(const kda_shape& s, const void* q, const void* k, const void* v, const void* la,
                            const void* beta, float* S, const int32_t* slots, int num_slots, void* o,
-                           cudaStream_t st) {
-  if (s.dk == 128 && s.dv == 128) return launch_decode<128, 128, TIO, TG>(s, q, k, v, la, beta, S, slots, num_slots, o, st);
-  if (s.dk == 64 && s.dv == 64) return launch_decode<64, 64, TIO, TG>(s, q, k, v, la, beta, S, slots, num_slots, o, st);
-  if (s.dk == 128 && s.dv == 64) return launch_decode<128, 64, TIO, TG>(s, q, k, v, la, beta, S, slots, num_slots, o, st);
-  return launch_decode<64, 128, TIO, TG>(s, q, k, v, la, beta, S, slots, num_slots, o, st);
+                           cudaStream_t st, const kda::RecProducer& pr, const kda::RecConsumer& cs) {
+  if (s.dk == 128 && s.dv == 128)
+    return launch_decode<128, 128, TIO, TG>(s, q, k, v, la, beta, S, slots, num_slots, o, st, pr, cs);
+  if (s.dk == 64 && s.dv == 64)
+    return launch_decode<64, 64, TIO, TG>(s, q, k, v, la, beta, S, slots, num_slots, o, st, pr, cs);
+  if (s.dk == 128 && s.dv == 64)
+    return launch_decode<128, 64, TIO, TG>(s, q, k, v, la, beta, S, slots, num_slots, o, st, pr, cs);
+  return launch_decode<64, 128, TIO, TG>(s, q, k, v, la, beta, S, slots, num_slots, o, st, pr, cs);
 }
 
 // Opt-in to large dynamic shared memory.  Set on every launch: the call is
@@ -374,8 +382,15 @@ kda_status chunk_fwd(const kda_shape* sp, const void* q, const void* k, const vo
 
   if (ep.gate && Ttot > 0 && (!aligned16(o) || !aligned16(ep.gate))) return KDA_ERR_ALIGN;
   bool fused = false;
-  if (pr.A_log && (!use_tc(s) || s.gate_dtype != KDA_BF16)) return KDA_ERR_UNSUPPORTED;
-  if (pr.A_log && Ttot > 0) {
+  if (pr.A_log && use_tc(s) && s.gate_dtype != KDA_BF16) return KDA_ERR_UNSUPPORTED;
+  kda::RecProducer rp;
+  rp.A_log = pr.A_log;
+  rp.dt_bias = pr.dt_bias;
+  kda::RecConsumer rc;  // the CUDA-core kernels apply the output epilogue themselves
+  rc.gate = ep.gate;
+  rc.norm_w = ep.norm_w;
+  rc.eps = ep.eps;
+  if (pr.A_log && use_tc(s) && Ttot > 0) {
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(log_alpha) || !aligned16(o) ||
         !aligned16(pr.dt_bias))
       return KDA_ERR_ALIGN;
@@ -391,15 +406,19 @@ kda_status chunk_fwd(const kda_shape* sp, const void* q, const void* k, const vo
       e = launch_prefill<float, false>(s, N, Ttot, q, k, v, log_alpha, beta, io, ep, pr, cu_seqlens, o, workspace,
                                        workspace_bytes, st, &fused);
   } else if (s.io_dtype == KDA_F32) {
+    fused = ep.gate != nullptr;
     if (s.gate_dtype == KDA_F32)
-      e = dispatch_recurrent_fwd<float, float>(s, N, q, k, v, log_alpha, beta, io, cu_seqlens, o, st);
+      e = dispatch_recurrent_fwd<float, float>(s, N, q, k, v, log_alpha, beta, io, cu_seqlens, o, st, rp, rc);
     else
-      e = dispatch_recurrent_fwd<float, __nv_bfloat16>(s, N, q, k, v, log_alpha, beta, io, cu_seqlens, o, st);
+      e = dispatch_recurrent_fwd<float, __nv_bfloat16>(s, N, q, k, v, log_alpha, beta, io, cu_seqlens, o, st,
+                                                           rp, rc);
   } else if (s.gate_dtype == KDA_F32) {
-    e = dispatch_recurrent_fwd<__nv_bfloat16, float>(s, N, q, k, v, log_alpha, beta, io, cu_seqlens, o, st);
+    fused = ep.gate != nullptr;
+    e = dispatch_recurrent_fwd<__nv_bfloat16, float>(s, N, q, k, v, log_alpha, beta, io, cu_seqlens, o, st, rp, rc);
   } else {
+    fused = ep.gate != nullptr;
     e = dispatch_recurrent_fwd<__nv_bfloat16, __nv_bfloat16>(s, N, q, k, v, log_alpha, beta, io, cu_seqlens, o,
-                                                             st);
+                                                             st, rp, rc);
   }
   if (e != KDA_OK || !ep.gate || fused || Ttot == 0) return e;
   const int64_t rows = Ttot * s.H;
@@ -411,7 +430,8 @@ kda_status chunk_fwd(const kda_shape* sp, const void* q, const void* k, const vo
 
 // Shared body of kda_decode_step and kda_decode_step_slots.
 kda_status decode_step(const kda_shape* sp, const void* q, const void* k, const void* v, const void* log_alpha,
-                       const void* beta, float* S, const int32_t* slots, int num_slots, void* o, void* stream) {
+                       const void* beta, float* S, const int32_t* slots, int num_slots, void* o, void* stream,
+                       const kda::RecProducer& pr = kda::RecProducer{}, const Epilogue& ep = Epilogue{}) {
   kda_status e = check_common(sp);
   if (e != KDA_OK) return e;
   const kda_shape& s = *sp;
@@ -420,15 +440,21 @@ kda_status decode_step(const kda_shape* sp, const void* q, const void* k, const 
   if (!token_ptrs_aligned(s, q, k, v, log_alpha, beta, o) || !aligned16(S) || !aligned(slots, 4))
     return KDA_ERR_ALIGN;
   if (static_cast<int64_t>(s.B) * s.H > 0x7fffffffLL) return KDA_ERR_SHAPE;
+  if (ep.gate && (!aligned(ep.gate, s.io_dtype == KDA_F32 ? 4 : 2) || !aligned(ep.norm_w, 4))) return KDA_ERR_ALIGN;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  kda::RecConsumer cs;  // the output epilogue, in the kernel
+  cs.gate = ep.gate;
+  cs.norm_w = ep.norm_w;
+  cs.eps = ep.eps;
   if (s.io_dtype == KDA_F32) {
     if (s.gate_dtype == KDA_F32)
-      return dispatch_decode<float, float>(s, q, k, v, log_alpha, beta, S, slots, num_slots, o, st);
-    return dispatch_decode<float, __nv_bfloat16>(s, q, k, v, log_alpha, beta, S, slots, num_slots, o, st);
+      return dispatch_decode<float, float>(s, q, k, v, log_alpha, beta, S, slots, num_slots, o, st, pr, cs);
+    return dispatch_decode<float, __nv_bfloat16>(s, q, k, v, log_alpha, beta, S, slots, num_slots, o, st, pr, cs);
   }
   if (s.gate_dtype == KDA_F32)
-    return dispatch_decode<__nv_bfloat16, float>(s, q, k, v, log_alpha, beta, S, slots, num_slots, o, st);
-  return dispatch_decode<__nv_bfloat16, __nv_bfloat16>(s, q, k, v, log_alpha, beta, S, slots, num_slots, o, st);
+    return dispatch_decode<__nv_bfloat16, float>(s, q, k, v, log_alpha, beta, S, slots, num_slots, o, st, pr, cs);
+  return dispatch_decode<__nv_bfloat16, __nv_bfloat16>(s, q, k, v, log_alpha, beta, S, slots, num_slots, o, st, pr,
+                                                       cs);
 }
 
 }  // namespace
@@ -518,6 +544,29 @@ kda_status kda_decode_step_slots(const kda_shape* sp, const void* q, const void*
   if (!state_slots) return KDA_ERR_NULL;
   if (num_slots <= 0) return KDA_ERR_SHAPE;
   return decode_step(sp, q, k, v, log_alpha, beta, state_pool, state_slots, num_slots, o, stream);
+}
+
+kda_status kda_decode_step_layer(const kda_shape* sp, const void* q, const void* k, const void* v,
+                                 const void* gate_f, const float* A_log, const float* dt_bias, const void* beta,
+                                 float* state, const int32_t* state_slots, int32_t num_slots, const void* out_gate,
+                                 const float* norm_weight, float eps, void* o, void* stream) {
+  if (!sp) return KDA_ERR_NULL;
+  if (!A_log || !dt_bias) return KDA_ERR_NULL;
+  if (!aligned(A_log, 4) || !aligned(dt_bias, 4)) return KDA_ERR_ALIGN;
+  if (state_slots && num_slots <= 0) return KDA_ERR_SHAPE;
+  Epilogue ep;
+  if (out_gate || norm_weight) {
+    if (!out_gate || !norm_weight) return KDA_ERR_NULL;
+    if (!(eps >= 0.f) || !(eps < 3.0e38f)) return KDA_ERR_ARGUMENT;
+    if (!aligned16(out_gate) || !aligned16(norm_weight)) return KDA_ERR_ALIGN;
+    ep.gate = out_gate;
+    ep.norm_w = norm_weight;
+    ep.eps = eps;
+  }
+  kda::RecProducer pr;
+  pr.A_log = A_log;
+  pr.dt_bias = dt_bias;
+  return decode_step(sp, q, k, v, gate_f, beta, state, state_slots, state_slots ? num_slots : 0, o, stream, pr, ep);
 }
 
 kda_status kda_check_device_error(void* stream) {

@@ -63,7 +63,6 @@ constexpr int NTHREADS = 384;
 constexpr int MAX_RING = 16;  // ring slots per state CTA (the host picks 2..16)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kSpan2 = 230.0f;  // largest chunk decay of the factorised path, log2 units
-constexpr float kQKNormEps = 1e-6f;  // epsilon of the producer's L2 normalisation of q and k
 
 // ---- ring slot: operands of one chunk as the state CTA's MMAs read them ----
 // Part A (Tb, -W'^T, the per-channel scales) feeds U and is released once U

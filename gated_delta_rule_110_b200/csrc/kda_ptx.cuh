@@ -373,6 +373,9 @@ __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src)
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
+// Epsilon of the producer steps' L2 normalisation of q and k: x / sqrt(sum x^2 + eps).
+constexpr float kQKNormEps = 1e-6f;
+
 // tanh(x) on the MUFU unit (approximate: about 2^-11 relative error).
 __device__ __forceinline__ float tanh_approx(float x) {
   float y;

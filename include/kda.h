@@ -52,7 +52,7 @@
 extern "C" {
 #endif
 
-#define KDA_ABI_VERSION 5
+#define KDA_ABI_VERSION 6
 
 typedef enum {
   KDA_OK = 0,
@@ -171,9 +171,10 @@ kda_status kda_chunk_fwd(const kda_shape* shape, const void* q, const void* k, c
  *   eps          >= 0, added to the mean square.
  * Everything else as kda_chunk_fwd, on every path.  The tensor-core prefill
  * applies the epilogue in its output warps where its state CTAs have time
- * to spare (short, many sequences), else, and on the CUDA-core paths, a
- * second kernel on `stream` applies it to o in place (reads o and g, writes
- * o).  KDA_FLAG_GATE_FUSED / KDA_FLAG_GATE_SEPARATE force either.  The
+ * to spare (short, many sequences), else a second kernel on `stream` applies
+ * it to o in place (reads o and g, writes o); KDA_FLAG_GATE_FUSED /
+ * KDA_FLAG_GATE_SEPARATE force either.  The CUDA-core paths apply it to each
+ * token's o in their kernel (fp32 io with the accurate expf).  The
  * sigmoid is computed as (1 + tanh(g/2)) / 2 with the hardware tanh
  * approximation: within about 2.5e-4 absolute.
  */
@@ -204,12 +205,13 @@ kda_status kda_chunk_fwd_gated(const kda_shape* shape, const void* q, const void
  *   dt_bias   [H, dk] fp32; 16-byte aligned.
  *   out_gate, norm_weight, eps   as kda_chunk_fwd_gated, or out_gate and
  *             norm_weight both NULL for no epilogue (one NULL: KDA_ERR_NULL).
- * Everything else as kda_chunk_fwd.  Only the tensor-core path (bf16 io and
- * gates, dk = dv = 128, no KDA_FLAG_PATH_RECURRENT) runs the producer steps:
- * other shapes return KDA_ERR_UNSUPPORTED.  softplus and exp are evaluated in
- * fp32 with the hardware 2^x and log2 approximations, and log alpha enters
- * the chunk's cumulative sum with 16 significant bits (relative error below
- * 2^-16; the bf16 log_alpha of kda_chunk_fwd carries 8).
+ * Everything else as kda_chunk_fwd, on every path.  On the tensor-core path
+ * gate_f must be bf16 (gate_dtype KDA_BF16, else KDA_ERR_UNSUPPORTED);
+ * softplus and exp are evaluated in fp32 with the hardware 2^x and log2
+ * approximations, and log alpha enters the chunk's cumulative sum with 16
+ * significant bits (relative error below 2^-16; the bf16 log_alpha of
+ * kda_chunk_fwd carries 8).  The CUDA-core paths (fp32 io, dk or dv = 64,
+ * KDA_FLAG_PATH_RECURRENT) evaluate them with the accurate expf / log1pf.
  */
 #define KDA_QK_NORM_EPS 1e-6f
 kda_status kda_chunk_fwd_layer(const kda_shape* shape, const void* q, const void* k, const void* v,
@@ -217,6 +219,22 @@ kda_status kda_chunk_fwd_layer(const kda_shape* shape, const void* q, const void
                                const float* S0, const int32_t* cu_seqlens, const void* out_gate,
                                const float* norm_weight, float eps, void* o, float* S_T, void* workspace,
                                size_t workspace_bytes, void* stream);
+
+/*
+ * kda_decode_step_layer -- kda_decode_step (or, with state_slots,
+ * kda_decode_step_slots) with the layer's producer steps in the kernel and
+ * the optional output epilogue, as kda_chunk_fwd_layer defines them: q, k
+ * raw [B, 1, H, dk]; gate_f [B, 1, H, dk] in the gate dtype; A_log [H] and
+ * dt_bias [H, dk] fp32 (4-byte aligned); state dense [B, H, dk, dv] fp32
+ * (state_slots NULL) or a pool of num_slots slots; out_gate [B, 1, H, dv]
+ * (io dtype, 16-byte aligned) and norm_weight [dv] fp32, or both NULL.  The
+ * decode kernel applies the epilogue to each o before storing it.  Every
+ * shape of kda_decode_step is supported.
+ */
+kda_status kda_decode_step_layer(const kda_shape* shape, const void* q, const void* k, const void* v,
+                                 const void* gate_f, const float* A_log, const float* dt_bias, const void* beta,
+                                 float* state, const int32_t* state_slots, int32_t num_slots, const void* out_gate,
+                                 const float* norm_weight, float eps, void* o, void* stream);
 
 /*
  * kda_chunk_fwd_noalloc -- kda_chunk_fwd for callers that cannot allocate.

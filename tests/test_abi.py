@@ -30,7 +30,7 @@ def test_library_loads_and_exports_every_declared_symbol():
     lib = kda.load_library()
     for name in declared_functions():
         assert hasattr(lib, name), name
-    assert kda.kda_abi_version() == 5
+    assert kda.kda_abi_version() == 6
 
 
 def test_status_strings():
@@ -200,10 +200,11 @@ def test_layer_prefill_host_validation():
     assert call_fwd_layer(tc_shape(), weight=FAKE) == -1
     assert call_fwd_layer(tc_shape(), gate=FAKE, weight=FAKE, eps=-1.0) == -10
     assert call_fwd_layer(tc_shape(), gate=FAKE + 2, weight=FAKE) == -4
-    # the producer steps run in the tensor-core kernel only
-    for shape in (tc_shape(io_dtype=0), tc_shape(gate_dtype=0), tc_shape(dk=64, dv=64),
-                  tc_shape(flags=kda.KDA_FLAG_PATH_RECURRENT)):
-        assert call_fwd_layer(shape) == -5
+    # the tensor-core kernel takes a bf16 gate projection only; the CUDA-core
+    # paths take any (they get as far as the launch)
+    assert call_fwd_layer(tc_shape(gate_dtype=0)) == -5
+    for shape in (tc_shape(io_dtype=0), tc_shape(dk=64, dv=64), tc_shape(flags=kda.KDA_FLAG_PATH_RECURRENT)):
+        assert call_fwd_layer(shape) in (-6, -7)
     assert call_fwd_layer(tc_shape(B=2, T=200)) in (-6, -7)
     assert call_fwd_layer(tc_shape(B=2, T=200), gate=FAKE, weight=FAKE) in (-6, -7)
 
@@ -213,3 +214,20 @@ def test_python_binding_refuses_cpu_tensors():
     x = torch.zeros(1, 4, 1, 64)
     with pytest.raises(ValueError):
         kda.kda_chunk_fwd(x, x, x, x, torch.zeros(1, 4, 1))
+
+
+def test_layer_decode_host_validation():
+    lib = kda.load_library()
+    vp = lambda x: None if x is None else ctypes.c_void_p(x)
+    f = vp(FAKE)
+    s1 = kda.make_shape(4, 1, 2, 128, 128)
+    call = lambda shape, A=FAKE, bias=FAKE, slots=None, n=0, gate=None, w=None, eps=1e-5: lib.kda_decode_step_layer(
+        ctypes.byref(shape), f, f, f, f, vp(A), vp(bias), f, f, vp(slots), n, vp(gate), vp(w), ctypes.c_float(eps),
+        f, None)
+    assert call(s1, A=None) == -1
+    assert call(s1, bias=None) == -1
+    assert call(s1, A=FAKE + 2) == -4
+    assert call(s1, slots=FAKE, n=0) == -2
+    assert call(s1, gate=FAKE) == -1
+    assert call(s1, gate=FAKE, w=FAKE, eps=-1.0) == -10
+    assert call(kda.make_shape(4, 2, 2, 128, 128)) == -2

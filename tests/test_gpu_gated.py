@@ -36,7 +36,7 @@ def _bounds(o, cu):
     return [(0, int(c[n]), int(c[n + 1])) for n in range(len(c) - 1)]
 
 
-def _check(x, gate, w, eps, o, S):
+def _check(x, gate, w, eps, o, S, tol=TOL):
     cu = None if x["cu_seqlens"] is None else x["cu_seqlens"].cpu().numpy()
     o_ref, S_ref = oracle.forward(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["S0"], cu_seqlens=cu)
     y_ref = oracle.output_gate(o_ref, gate, w, eps)
@@ -48,9 +48,9 @@ def _check(x, gate, w, eps, o, S):
             err = max(err, max_rel_l2_per_slice(y[b, a:e], y_ref[b, a:e], slice_axes=(1,)))
             err_w = max(err_w, max_rel_l2_per_window(y[b, a:e], y_ref[b, a:e]))
     err_S = max_rel_l2_per_slice(S.cpu().numpy(), S_ref, slice_axes=(0, 1))
-    assert err <= TOL, f"gated o rel-L2 {err:.3e} > {TOL}"
-    assert err_w <= TOL, f"gated o rel-L2 on a 64-token window {err_w:.3e} > {TOL}"
-    assert err_S <= TOL, f"S_T rel-L2 {err_S:.3e} > {TOL}"
+    assert err <= tol, f"gated o rel-L2 {err:.3e} > {tol}"
+    assert err_w <= tol, f"gated o rel-L2 on a 64-token window {err_w:.3e} > {tol}"
+    assert err_S <= tol, f"S_T rel-L2 {err_S:.3e} > {tol}"
     return err
 
 
@@ -95,15 +95,17 @@ def test_gated_gate_and_epsilon_ranges(scale, eps, mode):
     _check(x, gate, w, eps, o, S)
 
 
-@pytest.mark.parametrize("d,dtype", [(64, torch.float32), (128, torch.float32), (128, torch.bfloat16)])
-def test_gated_cuda_core_paths(d, dtype):
+@pytest.mark.parametrize("d,dtype,tol", [(64, torch.float32, 1e-4), (128, torch.float32, 1e-4),
+                                         (128, torch.bfloat16, TOL)])
+def test_gated_cuda_core_paths(d, dtype, tol):
     """fp32 io, dk = dv = 64, and the bf16 token-by-token recurrence: the
-    epilogue runs as its own pass over o."""
+    CUDA-core kernel applies the epilogue to each token's o (fp32 io with
+    the accurate exp, within the fp32 bound)."""
     lens = [5, 64, 77]
     x = gen.make_inputs(1, sum(lens), 2, d, d, dtype=dtype, seqlens=lens, seed=50)
     gate, w = gen.output_gate_inputs(x["v"].shape, dtype=dtype, seed=51)
     o, S = _run(x, gate, w, 1e-5, recurrent=(dtype == torch.bfloat16))
-    _check(x, gate, w, 1e-5, o, S)
+    _check(x, gate, w, 1e-5, o, S, tol)
 
 
 @pytest.mark.parametrize("mode", MODES)

@@ -136,3 +136,74 @@ def test_layer_sharded_single_rank_is_the_plain_call():
                                      x["cu_seqlens"], out_gate=gate, norm_weight=w)
     assert kda.kda_check_device_error() == 0
     assert torch.equal(o1, o2) and torch.equal(S1, S2)
+
+
+# ---------------------------------------------------------------- CUDA-core paths and decode
+@pytest.mark.parametrize("d,dtype,tol", [(64, torch.float32, 1e-4), (128, torch.float32, 1e-4),
+                                         (128, torch.bfloat16, TOL)])
+def test_layer_cuda_core_paths(d, dtype, tol):
+    """fp32 io, dk = dv = 64, and the bf16 token-by-token recurrence run the
+    producer steps in the CUDA-core kernel (fp32 keeps its 1e-4 bound)."""
+    lens = [5, 64, 77]
+    x = gen.make_layer_inputs(1, sum(lens), 2, d, d, dtype=dtype, seqlens=lens, seed=72)
+    o, S = _run(x, recurrent=(dtype == torch.bfloat16))
+    cu = x["cu_seqlens"].numpy()
+    o_ref, S_ref = oracle.forward_layer(x["q"], x["k"], x["v"], x["f"], x["A_log"], x["dt_bias"], x["beta"], x["S0"],
+                                        cu_seqlens=cu, qk_eps=1e-6)
+    y = o.float().cpu().numpy()
+    c = [int(v) for v in cu]
+    err = max(max_rel_l2_per_slice(y[0, c[n]:c[n + 1]], o_ref[0, c[n]:c[n + 1]], slice_axes=(1,))
+              for n in range(len(lens)))
+    assert err <= tol
+    assert max_rel_l2_per_slice(S.cpu().numpy(), S_ref, slice_axes=(0, 1)) <= tol
+
+
+def _decode_ref(xs, S, gate=None, w=None, eps=1e-5):
+    q, k = oracle.l2norm(xs["q"], 1e-6), oracle.l2norm(xs["k"], 1e-6)
+    la = oracle.decay_gate(xs["f"], xs["A_log"], xs["dt_bias"])
+    o, S1 = oracle.decode(q, k, xs["v"], la, xs["beta"], S)
+    if gate is not None:
+        o = oracle.output_gate(o, gate, w, eps)
+    return o, S1
+
+
+@pytest.mark.parametrize("d,dtype,tol", [(128, torch.bfloat16, TOL), (64, torch.float32, 1e-4)])
+@pytest.mark.parametrize("epilogue", [False, True])
+def test_decode_layer_dense_steps(d, dtype, tol, epilogue):
+    N, H = 6, 3
+    S = gen.decode_state(N, H, d, d, seed=81).cuda()
+    S_ref = S.cpu().double().numpy()
+    for step in range(3):
+        x = gen.make_layer_inputs(N, 1, H, d, d, dtype=dtype, seed=82 + step)
+        xs = {kk: x[kk][:, 0] for kk in ("q", "k", "v", "f", "beta")}
+        xs["A_log"], xs["dt_bias"] = x["A_log"], x["dt_bias"]
+        gate, w = gen.output_gate_inputs((N, H, d), dtype=dtype, seed=90 + step) if epilogue else (None, None)
+        o = kda.kda_decode_step_layer(xs["q"].cuda(), xs["k"].cuda(), xs["v"].cuda(), xs["f"].cuda(),
+                                      xs["A_log"].cuda(), xs["dt_bias"].cuda(), xs["beta"].cuda(), S,
+                                      out_gate=None if gate is None else gate.cuda(),
+                                      norm_weight=None if w is None else w.cuda())
+        assert kda.kda_check_device_error() == 0
+        o_ref, S_ref = _decode_ref(xs, S_ref, gate, w)
+        assert max_rel_l2_per_slice(o.float().cpu().numpy(), o_ref, slice_axes=(0, 1)) <= tol
+        assert max_rel_l2_per_slice(S.cpu().numpy(), S_ref, slice_axes=(0, 1)) <= tol
+
+
+def test_decode_layer_slots_equal_dense():
+    """Through pool slots (permuted, one padding entry) the step matches the
+    dense call on the gathered rows, bit for bit."""
+    N, H, d = 5, 2, 128
+    pool = gen.decode_state(8, H, d, d, seed=91).cuda()
+    slots = torch.tensor([6, 1, -1, 3, 0], dtype=torch.int32, device="cuda")
+    x = gen.make_layer_inputs(N, 1, H, d, d, seed=92, device="cuda")
+    args = [x[kk][:, 0] for kk in ("q", "k", "v", "f")] + [x["A_log"], x["dt_bias"], x["beta"][:, 0]]
+    dense = torch.zeros((N, H, d, d), device="cuda")
+    live = [0, 1, 3, 4]
+    dense[live] = pool[slots[live].long()]
+    o_d = kda.kda_decode_step_layer(*args, dense)
+    pool2 = pool.clone()
+    o_s = kda.kda_decode_step_layer(*args, pool2, state_slots=slots)
+    assert kda.kda_check_device_error() == 0
+    assert torch.equal(o_s[live], o_d[live])
+    assert torch.equal(pool2[slots[live].long()], dense[live])
+    untouched = [i for i in range(8) if i not in (6, 1, 3, 0)]
+    assert torch.equal(pool2[untouched], pool[untouched])
