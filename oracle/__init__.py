@@ -53,6 +53,10 @@ def _load():
         lib.kda_oracle_mutation_count.restype = ctypes.c_int
         lib.kda_oracle_output_gate.argtypes = [ctypes.c_int64, ctypes.c_int, dp, dp, dp, ctypes.c_double, dp]
         lib.kda_oracle_output_gate.restype = ctypes.c_int
+        ip = ctypes.POINTER(ctypes.c_int64)
+        lib.kda_oracle_backward.argtypes = [ctypes.c_int, ip, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                            dp, dp, dp, dp, dp, dp, dp, dp, dp, dp, dp, dp, dp, dp]
+        lib.kda_oracle_backward.restype = ctypes.c_int
         lib.kda_oracle_l2norm.argtypes = [ctypes.c_int64, ctypes.c_int, dp, ctypes.c_double, dp]
         lib.kda_oracle_l2norm.restype = ctypes.c_int
         lib.kda_oracle_decay_gate.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, dp, dp, dp, dp]
@@ -171,3 +175,35 @@ def forward_layer(q, k, v, f, A_log, dt_bias, beta, S0=None, cu_seqlens=None, qk
     if out_gate is not None:
         o = output_gate(o, out_gate, norm_weight, eps)
     return o, S
+
+
+def backward(q, k, v, log_alpha, beta, S0=None, dO=None, dS_T=None, cu_seqlens=None):
+    """Gradients of the operator in fp64 by hand-written reverse-mode
+    differentiation of the token recurrence (kda_oracle.c,
+    kda_oracle_backward).  Shapes as forward; dO like o, dS_T like S_T.
+    Returns (dq, dk, dv, dlog_alpha, dbeta, dS0)."""
+    q, k, v, la, b = (_f64(x) for x in (q, k, v, log_alpha, beta))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if cu_seqlens is None:
+        cu = np.arange(B + 1, dtype=np.int64) * T
+    else:
+        if B != 1:
+            raise ValueError("packed input needs B == 1")
+        cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int64))
+    N = len(cu) - 1
+    s0 = None if S0 is None else _f64(S0).reshape(N, H, dk, dv)
+    gO = None if dO is None else _f64(dO).reshape(B * T, H, dv)
+    gS = None if dS_T is None else _f64(dS_T).reshape(N, H, dk, dv)
+    dq, dk_, dla = (np.zeros((B * T, H, dk)) for _ in range(3))
+    dv_ = np.zeros((B * T, H, dv))
+    db = np.zeros((B * T, H))
+    dS0 = np.zeros((N, H, dk, dv))
+    opt = lambda a: _ptr(a) if a is not None else None
+    rc = _load().kda_oracle_backward(
+        N, cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), H, dk, dv, _ptr(q), _ptr(k), _ptr(v), _ptr(la),
+        _ptr(b), opt(s0), opt(gO), opt(gS), _ptr(dq), _ptr(dk_), _ptr(dv_), _ptr(dla), _ptr(db), _ptr(dS0))
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments")
+    r = lambda a, last: a.reshape(B, T, H, *last)
+    return (r(dq, (dk,)), r(dk_, (dk,)), r(dv_, (dv,)), r(dla, (dk,)), db.reshape(B, T, H), dS0)

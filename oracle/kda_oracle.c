@@ -320,3 +320,135 @@ int kda_oracle_decay_gate(int64_t tokens, int H, int dk, const double* f, const 
     }
   return 0;
 }
+
+/*
+ * kda_oracle_backward -- gradients of the operator (no page prints them; the
+ * chunkwise algorithm section of the "Kimi Linear" summary mentions the UT
+ * transform's use in training).  Reverse-mode differentiation of the token
+ * recurrence above, written out by hand, per (sequence, head):
+ *
+ *   forward, token t (S_prev the state before it):
+ *     S~ = Diag(alpha) S_prev,  u = v - S~^T k,  S = S~ + beta k u^T,  o = S^T q
+ *   backward, with dS the gradient reaching S_t from later tokens (dS_T at
+ *   the end) and do = dL/do_t:
+ *     dq   = S do                      dS  += q do^T
+ *     dbeta = k^T dS u                 du   = beta dS^T k
+ *     dk   = beta dS u - S~ du         dv   = du
+ *     dS~  = dS - k du^T
+ *     dlog_alpha[i] = sum_j dS~[i][j] S~[i][j]     (d alpha = alpha d log alpha)
+ *     dS_prev = Diag(alpha) dS~
+ *   and dS0 = the gradient reaching the initial state.
+ *
+ * Layouts as kda_oracle_forward; dO like o, dS_T like S_T (either may be
+ * NULL: no gradient from it).  Outputs dq, dk, dlog_alpha like q; dv like v;
+ * dbeta like beta; dS0 like S0 (always written).  The forward states are
+ * recomputed and kept for the whole sequence (test sizes only).
+ */
+int kda_oracle_backward(int n_seqs, const int64_t* cu_seqlens, int H, int dk, int dv,
+                        const double* q, const double* k, const double* v, const double* log_alpha,
+                        const double* beta, const double* S0, const double* dO, const double* dS_T,
+                        double* dq, double* dk_out, double* dv_out, double* dla, double* dbeta, double* dS0)
+{
+  if (n_seqs < 0 || H <= 0 || dk <= 0 || dv <= 0 || !cu_seqlens) return -1;
+  const size_t dd = (size_t)dk * dv;
+  for (int n = 0; n < n_seqs; ++n) {
+    const int64_t t0 = cu_seqlens[n], t1 = cu_seqlens[n + 1];
+    if (t1 < t0) return -1;
+    const int64_t L = t1 - t0;
+    for (int h = 0; h < H; ++h) {
+      /* states[i] = state after i tokens of this sequence (states[0] = S0) */
+      double* states = (double*)calloc((size_t)(L + 1) * dd, sizeof(double));
+      double* dS = (double*)calloc(dd, sizeof(double));
+      double* St = (double*)malloc(dd * sizeof(double));
+      double* u = (double*)malloc((size_t)dv * sizeof(double));
+      double* du = (double*)malloc((size_t)dv * sizeof(double));
+      if (!states || !dS || !St || !u || !du) {
+        free(states); free(dS); free(St); free(u); free(du);
+        return -1;
+      }
+      if (S0) memcpy(states, S0 + ((size_t)n * H + h) * dd, dd * sizeof(double));
+      for (int64_t i = 0; i < L; ++i) {
+        const int64_t row = (t0 + i) * H + h;
+        const double* kt = k + row * dk;
+        const double* vt = v + row * dv;
+        const double b = beta[row];
+        const double* Sp = states + (size_t)i * dd;
+        double* Sn = states + (size_t)(i + 1) * dd;
+        for (int a = 0; a < dk; ++a) {
+          const double al = exp(log_alpha[row * dk + a]);
+          for (int j = 0; j < dv; ++j) St[a * dv + j] = al * Sp[a * dv + j];
+        }
+        for (int j = 0; j < dv; ++j) {
+          double r = 0.0;
+          for (int a = 0; a < dk; ++a) r += St[a * dv + j] * kt[a];
+          u[j] = vt[j] - r;
+        }
+        for (int a = 0; a < dk; ++a)
+          for (int j = 0; j < dv; ++j) Sn[a * dv + j] = St[a * dv + j] + b * kt[a] * u[j];
+      }
+      if (dS_T) memcpy(dS, dS_T + ((size_t)n * H + h) * dd, dd * sizeof(double));
+      for (int64_t i = L - 1; i >= 0; --i) {
+        const int64_t row = (t0 + i) * H + h;
+        const double* qt = q + row * dk;
+        const double* kt = k + row * dk;
+        const double* vt = v + row * dv;
+        const double b = beta[row];
+        const double* Sp = states + (size_t)i * dd;
+        const double* Sn = states + (size_t)(i + 1) * dd;
+        /* o = S^T q */
+        for (int a = 0; a < dk; ++a) {
+          double g = 0.0;
+          if (dO)
+            for (int j = 0; j < dv; ++j) g += Sn[a * dv + j] * dO[row * dv + j];
+          dq[row * dk + a] = g;
+        }
+        if (dO)
+          for (int a = 0; a < dk; ++a)
+            for (int j = 0; j < dv; ++j) dS[a * dv + j] += qt[a] * dO[row * dv + j];
+        /* recompute S~ and u of this token */
+        for (int a = 0; a < dk; ++a) {
+          const double al = exp(log_alpha[row * dk + a]);
+          for (int j = 0; j < dv; ++j) St[a * dv + j] = al * Sp[a * dv + j];
+        }
+        for (int j = 0; j < dv; ++j) {
+          double r = 0.0;
+          for (int a = 0; a < dk; ++a) r += St[a * dv + j] * kt[a];
+          u[j] = vt[j] - r;
+        }
+        /* S = S~ + beta k u^T */
+        double db = 0.0;
+        for (int a = 0; a < dk; ++a)
+          for (int j = 0; j < dv; ++j) db += kt[a] * dS[a * dv + j] * u[j];
+        dbeta[row] = db;
+        for (int j = 0; j < dv; ++j) {
+          double r = 0.0;
+          for (int a = 0; a < dk; ++a) r += dS[a * dv + j] * kt[a];
+          du[j] = b * r;
+          dv_out[row * dv + j] = du[j];  /* u = v - S~^T k */
+        }
+        for (int a = 0; a < dk; ++a) {
+          double g1 = 0.0, g2 = 0.0;
+          for (int j = 0; j < dv; ++j) {
+            g1 += dS[a * dv + j] * u[j];
+            g2 += St[a * dv + j] * du[j];
+          }
+          dk_out[row * dk + a] = b * g1 - g2;
+        }
+        /* dS~ = dS - k du^T; then through the decay */
+        for (int a = 0; a < dk; ++a) {
+          const double al = exp(log_alpha[row * dk + a]);
+          double gl = 0.0;
+          for (int j = 0; j < dv; ++j) {
+            const double g = dS[a * dv + j] - kt[a] * du[j];
+            gl += g * St[a * dv + j];
+            dS[a * dv + j] = al * g;
+          }
+          dla[row * dk + a] = gl;
+        }
+      }
+      if (dS0) memcpy(dS0 + ((size_t)n * H + h) * dd, dS, dd * sizeof(double));
+      free(states); free(dS); free(St); free(u); free(du);
+    }
+  }
+  return 0;
+}
