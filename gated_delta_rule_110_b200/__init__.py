@@ -49,7 +49,8 @@ _STATUS_NAMES = {
 }
 
 EXPORTED_SYMBOLS = (
-    "kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_chunk_fwd_gated", "kda_chunk_fwd_layer",
+    "kda_chunk_fwd_workspace_size", "kda_prefill_plan", "kda_chunk_fwd", "kda_chunk_fwd_gated",
+    "kda_chunk_fwd_layer",
     "kda_chunk_fwd_noalloc",
     "kda_chunk_fwd_slots",
     "kda_decode_step", "kda_decode_step_slots", "kda_decode_step_layer", "kda_check_device_error", "kda_status_string",
@@ -104,6 +105,8 @@ def load_library(build_if_missing: bool = True):
     lib.kda_decode_step_layer.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_int32, vp, vp,
                                           ctypes.c_float, vp, vp]
     lib.kda_decode_step_layer.restype = ctypes.c_int
+    lib.kda_prefill_plan.argtypes = [sp, ctypes.c_int32, ctypes.POINTER(PrefillPlanInfo)]
+    lib.kda_prefill_plan.restype = ctypes.c_int
     lib.kda_chunk_fwd_noalloc.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.kda_chunk_fwd_noalloc.restype = ctypes.c_int
     lib.kda_chunk_fwd_slots.argtypes = [sp, vp, vp, vp, vp, vp, vp, ctypes.c_int32, vp, vp, vp, vp, vp,
@@ -327,6 +330,24 @@ def kda_decode_step_layer(q, k, v, gate_f, A_log, dt_bias, beta, state, *, state
     if rc != KDA_OK:
         raise KdaError(rc, "kda_decode_step_layer")
     return o
+
+
+class PrefillPlanInfo(ctypes.Structure):
+    """kda_prefill_plan_info (include/kda.h)."""
+    _fields_ = [("state_ctas", ctypes.c_int32), ("grid_ctas", ctypes.c_int32), ("ring_depth", ctypes.c_int32),
+                ("fuse_output_gate", ctypes.c_int32), ("workspace_bytes", ctypes.c_uint64),
+                ("min_workspace_bytes", ctypes.c_uint64)]
+
+
+def kda_prefill_plan(shape, num_sms: int = 0) -> dict:
+    """The tensor-core prefill's plan for ``shape`` (a kda_shape) on a device
+    with ``num_sms`` SMs (0: the current device): state / transform CTA split,
+    ring depth, output-epilogue placement and workspace sizes."""
+    info = PrefillPlanInfo()
+    rc = load_library().kda_prefill_plan(ctypes.byref(shape), int(num_sms), ctypes.byref(info))
+    if rc != KDA_OK:
+        raise KdaError(rc, "kda_prefill_plan")
+    return {name: getattr(info, name) for name, _ in PrefillPlanInfo._fields_}
 
 
 def kda_chunk_fwd_noalloc(q, k, v, log_alpha, beta, S0, cu_seqlens, o, S_T, *, chunk: int = 64, stream=None,

@@ -340,6 +340,29 @@ size_t kda_chunk_fwd_workspace_size(const kda_shape* sp) {
   return plan_prefill(s, N, device_sm_count()).bytes;
 }
 
+kda_status kda_prefill_plan(const kda_shape* sp, int32_t num_sms, kda_prefill_plan_info* out) {
+  if (!out) return KDA_ERR_NULL;
+  const kda_status e = check_common(sp);
+  if (e != KDA_OK) return e;
+  const kda_shape& s = *sp;
+  if (!use_tc(s)) return KDA_ERR_UNSUPPORTED;
+  if (num_sms <= 0) num_sms = device_sm_count();
+  if (num_sms <= 0) return KDA_ERR_CUDA;
+  const bool packed = s.n_seqs > 0 && s.B == 1;
+  const int64_t N = packed ? s.n_seqs : s.B;
+  const PrefillPlan pl = plan_prefill(s, N, num_sms);
+  if (pl.R <= 0) return KDA_ERR_SHAPE;
+  out->state_ctas = pl.R;
+  out->grid_ctas = pl.grid;
+  out->ring_depth = pl.nring(pl.bytes);
+  out->fuse_output_gate = (s.flags & KDA_FLAG_GATE_FUSED) != 0u     ? 1
+                          : (s.flags & KDA_FLAG_GATE_SEPARATE) != 0u ? 0
+                                                                     : (pl.fuse_gate ? 1 : 0);
+  out->workspace_bytes = pl.bytes;
+  out->min_workspace_bytes = pl.min_bytes;
+  return KDA_OK;
+}
+
 }  // extern "C"
 
 namespace {

@@ -52,7 +52,7 @@
 extern "C" {
 #endif
 
-#define KDA_ABI_VERSION 6
+#define KDA_ABI_VERSION 7
 
 typedef enum {
   KDA_OK = 0,
@@ -119,6 +119,26 @@ typedef struct kda_shape {
  * the library rejects; kda_chunk_fwd then reports the reason.
  */
 size_t kda_chunk_fwd_workspace_size(const kda_shape* shape);
+
+/*
+ * kda_prefill_plan -- how the tensor-core prefill would run `shape` on a
+ * device with num_sms SMs (num_sms <= 0: the current device's count): the
+ * split of its one-CTA-per-SM grid into state CTAs (one serial chain of
+ * chunks each, chains i, i + R, ...) and transform CTAs, the preferred
+ * operand-ring depth per state CTA, whether kda_chunk_fwd_gated would fuse
+ * the output epilogue (honouring KDA_FLAG_GATE_*), and the workspace sizes.
+ * Host-only (with num_sms > 0 it touches no device).  KDA_ERR_UNSUPPORTED
+ * for shapes the tensor-core path does not take.
+ */
+typedef struct kda_prefill_plan_info {
+  int32_t state_ctas;        /* R                                                 */
+  int32_t grid_ctas;         /* all CTAs of the launch                            */
+  int32_t ring_depth;        /* operand-ring slots per state CTA (preferred)      */
+  int32_t fuse_output_gate;  /* 1: in the prefill kernel; 0: a separate pass      */
+  uint64_t workspace_bytes;      /* = kda_chunk_fwd_workspace_size on that device */
+  uint64_t min_workspace_bytes;  /* the smallest workspace accepted (2-slot ring)  */
+} kda_prefill_plan_info;
+kda_status kda_prefill_plan(const kda_shape* shape, int32_t num_sms, kda_prefill_plan_info* out);
 
 /*
  * kda_chunk_fwd -- chunkwise-parallel prefill ("Algoritmo paralelo por

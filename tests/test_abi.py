@@ -30,7 +30,7 @@ def test_library_loads_and_exports_every_declared_symbol():
     lib = kda.load_library()
     for name in declared_functions():
         assert hasattr(lib, name), name
-    assert kda.kda_abi_version() == 6
+    assert kda.kda_abi_version() == 7
 
 
 def test_status_strings():
@@ -231,3 +231,41 @@ def test_layer_decode_host_validation():
     assert call(s1, gate=FAKE) == -1
     assert call(s1, gate=FAKE, w=FAKE, eps=-1.0) == -10
     assert call(kda.make_shape(4, 2, 2, 128, 128)) == -2
+
+
+def test_prefill_plan_on_a_148_sm_device():
+    """The host's plan for the benchmark workloads on a 148-SM B200: state /
+    transform split, where the output epilogue goes, ring depth and
+    workspace (host-only: no device is touched with num_sms given)."""
+    from gated_delta_rule_110_b200 import inputs as gen
+    def plan(name, flags=0):
+        w = gen.workload(name)
+        n = 0 if w.seqlens is None else len(w.seqlens)
+        return kda.kda_prefill_plan(kda.make_shape(w.B, w.T, w.H, w.dk, w.dv, 64, n, 1, 1, flags), 148)
+    pre, var, lng = plan("prefill"), plan("varlen"), plan("long")
+    # 64 chains: one per state CTA, the other 84 CTAs transform (state side 1 chain, transform 128 / 84)
+    assert (pre["state_ctas"], pre["grid_ctas"]) == (64, 148)
+    # 256 chains: R balances ceil(256 / R) against 512 / (148 - R)
+    assert var["state_ctas"] == 52
+    assert lng["state_ctas"] == 32
+    # the epilogue is fused where the transform side bounds the call
+    assert pre["fuse_output_gate"] == 1 and var["fuse_output_gate"] == 1 and lng["fuse_output_gate"] == 0
+    assert plan("long", kda.KDA_FLAG_GATE_FUSED)["fuse_output_gate"] == 1
+    assert plan("prefill", kda.KDA_FLAG_GATE_SEPARATE)["fuse_output_gate"] == 0
+    for p in (pre, var, lng):
+        slot_bytes = p["state_ctas"] * 66560
+        assert 4 <= p["ring_depth"] <= 16
+        assert p["workspace_bytes"] >= p["ring_depth"] * slot_bytes
+        assert p["min_workspace_bytes"] < p["workspace_bytes"]
+        assert p["ring_depth"] == 4 or p["ring_depth"] * slot_bytes <= 48 << 20
+    # overrides through the flags
+    assert plan("prefill", kda.tuning_flags(16, 0))["state_ctas"] == 16
+    assert plan("prefill", kda.tuning_flags(0, 100))["grid_ctas"] == 100
+
+
+def test_prefill_plan_refuses_other_paths():
+    lib = kda.load_library()
+    info = kda.PrefillPlanInfo()
+    assert lib.kda_prefill_plan(ctypes.byref(tc_shape(io_dtype=0)), 148, ctypes.byref(info)) == -5
+    assert lib.kda_prefill_plan(ctypes.byref(tc_shape()), 148, None) == -1
+    assert lib.kda_prefill_plan(None, 148, ctypes.byref(info)) == -1
