@@ -182,3 +182,22 @@ def kda_chunk_fwd_layer_sharded(q, k, v, gate_f, A_log, dt_bias, beta, S0=None, 
         return fwd(lq, lk, lv, lf, lb, ls0, lcu, lgate, lA, lbias, norm_weight=norm_weight, eps=eps)
     return kda_chunk_fwd_sharded(q, k, v, gate_f, beta, S0, cu_seqlens, group=group, fwd=shard_fwd, gather=gather,
                                  token_extras=tok, head_extras=(A_log, dt_bias))
+
+
+def kda_chunk_fwd_gated_sharded(q, k, v, log_alpha, beta, out_gate, norm_weight, S0=None, cu_seqlens=None, *,
+                                eps: float = 1e-5, group=None, fwd=None, gather: bool = True):
+    """kda_chunk_fwd_gated (prefill, then the per-head RMSNorm and output
+    gate) split across the ranks of ``group``: out_gate is sliced like q.
+    ``fwd`` (default: the library's kda_chunk_fwd_gated) is called as
+    fwd(q, k, v, log_alpha, beta, S0, cu_seqlens, out_gate, norm_weight=...,
+    eps=...)."""
+    if fwd is None:
+        from . import kda_chunk_fwd_gated
+
+        def fwd(lq, lk, lv, la, lb, ls0, lcu, lgate, norm_weight=None, eps=1e-5):
+            return kda_chunk_fwd_gated(lq, lk, lv, la, lb, lgate, norm_weight, ls0, lcu, eps=eps)
+
+    def shard_fwd(lq, lk, lv, la, lb, ls0, lcu, lgate):
+        return fwd(lq, lk, lv, la, lb, ls0, lcu, lgate, norm_weight=norm_weight, eps=eps)
+    return kda_chunk_fwd_sharded(q, k, v, log_alpha, beta, S0, cu_seqlens, group=group, fwd=shard_fwd,
+                                 gather=gather, token_extras=(out_gate,))

@@ -152,3 +152,36 @@ def test_two_gloo_ranks_layer_path(tmp_path, name, kind):
         assert got["kind"] == kind
         assert torch.equal(got["o"], o_ref), f"rank {r}: o differs"
         assert torch.equal(got["S"], S_ref), f"rank {r}: S_T differs"
+
+
+def _oracle_gated_fwd(q, k, v, la, beta, S0, cu, gate, norm_weight=None, eps=1e-5):
+    import oracle
+    o, S = oracle.forward(q, k, v, la, beta, S0, cu_seqlens=None if cu is None else cu.numpy())
+    return torch.from_numpy(oracle.output_gate(o, gate, norm_weight, eps)), torch.from_numpy(S)
+
+
+def _gated_rank_main(rank, world, port, out_dir):
+    import torch.distributed as dist
+    from gated_delta_rule_110_b200.shard import kda_chunk_fwd_gated_sharded
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world)
+    try:
+        x = _case("packed")
+        gate, w = gen.output_gate_inputs(x["v"].shape, dtype=torch.float32, seed=74)
+        o, S, plan = kda_chunk_fwd_gated_sharded(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], gate, w, x["S0"],
+                                                 x["cu_seqlens"], fwd=_oracle_gated_fwd)
+        torch.save({"o": o, "S": S}, os.path.join(out_dir, f"r{rank}.pt"))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_gated_path(tmp_path):
+    world = 2
+    mp.start_processes(_gated_rank_main, args=(world, _free_port(), str(tmp_path)), nprocs=world,
+                       start_method="spawn", join=True)
+    x = _case("packed")
+    gate, w = gen.output_gate_inputs(x["v"].shape, dtype=torch.float32, seed=74)
+    o_ref, S_ref = _oracle_gated_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["S0"], x["cu_seqlens"],
+                                     gate, norm_weight=w)
+    for r in range(world):
+        got = torch.load(tmp_path / f"r{r}.pt")
+        assert torch.equal(got["o"], o_ref) and torch.equal(got["S"], S_ref)
