@@ -17,14 +17,18 @@ Entry points (same names as the C ABI):
 * ``kda_decode_step_layer(q, k, v, gate_f, A_log, dt_bias, beta, state, ...)`` one
   decode step with the layer's producer steps (and optional output epilogue)
 * ``kda_chunk_fwd_gated(q, k, v, log_alpha, beta, out_gate, norm_weight, ...)``
-  prefill with the per-head RMSNorm and sigmoid output gate fused -> ``(o', S_T)``
+  prefill followed by the per-head RMSNorm and sigmoid output gate -> ``(o', S_T)``
 * ``kda_chunk_fwd_slots(q, k, v, log_alpha, beta, state_pool, state_slots,
   has_initial_state=None, cu_seqlens=None)`` prefill reading and writing the
   states in place in a slot-indexed pool -> ``o``
 * ``kda_decode_step_slots(q, k, v, log_alpha, beta, state_pool, state_slots)``
   decode step on a slot-indexed pool -> ``o``
-* ``kda_chunk_fwd_workspace_size(...)``, ``kda_check_device_error()``,
-  ``kda_status_string(code)``, ``kda_abi_version()``
+* ``kda_chunk_fwd_noalloc(...)`` kda_chunk_fwd on the library's own scratch array
+* ``kda_chunk_fwd_workspace_size(...)``, ``kda_prefill_plan(shape, num_sms)``,
+  ``kda_check_device_error()``, ``kda_status_string(code)``, ``kda_abi_version()``
+
+Sharded variants (one batch across the ranks of a process group) are in
+``gated_delta_rule_110_b200.shard``.
 """
 from __future__ import annotations
 
