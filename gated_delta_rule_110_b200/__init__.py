@@ -231,13 +231,13 @@ def kda_chunk_fwd_gated(q, k, v, log_alpha, beta, out_gate, norm_weight, S0=None
     "auto" (the library decides), "fused" (in the tensor-core kernel's output
     warps) or "separate" (a pass over o after the prefill)."""
     import torch
-    _need_cuda(q, k, v, log_alpha, beta, out_gate, norm_weight, S0, cu_seqlens, o, S_T, workspace)
     if out_gate.shape != v.shape or out_gate.dtype != v.dtype:
         raise ValueError("out_gate must have the shape and dtype of v")
     if norm_weight.dtype != torch.float32 or norm_weight.numel() != v.shape[-1]:
         raise ValueError("norm_weight must be a float32 tensor of dv values")
     if gate_mode not in _GATE_MODES:
         raise ValueError(f"gate_mode must be one of {sorted(_GATE_MODES)}")
+    _need_cuda(q, k, v, log_alpha, beta, out_gate, norm_weight, S0, cu_seqlens, o, S_T, workspace)
     shape = _shape_of(q, v, log_alpha, cu_seqlens, chunk, validate, recurrent, state_ctas, grid_ctas)
     shape.flags |= _GATE_MODES[gate_mode]
     N = shape.B if cu_seqlens is None else shape.n_seqs
@@ -267,7 +267,6 @@ def kda_chunk_fwd_layer(q, k, v, gate_f, A_log, dt_bias, beta, S0=None, cu_seqle
     and, with ``out_gate`` / ``norm_weight``, its output epilogue
     (include/kda.h, kda_chunk_fwd_layer).  Returns (o, S_T)."""
     import torch
-    _need_cuda(q, k, v, gate_f, A_log, dt_bias, beta, S0, cu_seqlens, out_gate, norm_weight, o, S_T, workspace)
     H, dk = q.shape[2], q.shape[3]
     if gate_f.shape != q.shape or gate_f.dtype != q.dtype:
         raise ValueError("gate_f must have the shape and dtype of q")
@@ -282,6 +281,7 @@ def kda_chunk_fwd_layer(q, k, v, gate_f, A_log, dt_bias, beta, S0=None, cu_seqle
             raise ValueError("norm_weight must be a float32 tensor of dv values")
     if gate_mode not in _GATE_MODES:
         raise ValueError(f"gate_mode must be one of {sorted(_GATE_MODES)}")
+    _need_cuda(q, k, v, gate_f, A_log, dt_bias, beta, S0, cu_seqlens, out_gate, norm_weight, o, S_T, workspace)
     shape = _shape_of(q, v, gate_f, cu_seqlens, chunk, validate, recurrent, state_ctas, grid_ctas)
     shape.flags |= _GATE_MODES[gate_mode]
     N = shape.B if cu_seqlens is None else shape.n_seqs
@@ -309,7 +309,6 @@ def kda_decode_step_layer(q, k, v, gate_f, A_log, dt_bias, beta, state, *, state
     is updated in place (dense rows, or pool slots with ``state_slots``).
     Inputs [N, H, d] (one token per sequence) or [N, 1, H, d]; returns o."""
     import torch
-    _need_cuda(q, k, v, gate_f, A_log, dt_bias, beta, state, state_slots, out_gate, norm_weight, o)
     if q.dim() == 3:
         q, k, v, gate_f = (t.unsqueeze(1) for t in (q, k, v, gate_f))
         beta = beta.unsqueeze(1)
@@ -320,6 +319,9 @@ def kda_decode_step_layer(q, k, v, gate_f, A_log, dt_bias, beta, state, *, state
         raise ValueError("out_gate and norm_weight go together")
     if A_log.dtype != torch.float32 or dt_bias.dtype != torch.float32:
         raise ValueError("A_log and dt_bias must be float32")
+    if A_log.numel() != H or dt_bias.numel() != H * dk:
+        raise ValueError("A_log must have H values and dt_bias H * dk")
+    _need_cuda(q, k, v, gate_f, A_log, dt_bias, beta, state, state_slots, out_gate, norm_weight, o)
     shape = _shape_of(q, v, gate_f, None, 64, False)
     if o is None:
         o = torch.empty((N, H, v.shape[-1]), dtype=v.dtype, device=v.device)

@@ -269,3 +269,29 @@ def test_prefill_plan_refuses_other_paths():
     assert lib.kda_prefill_plan(ctypes.byref(tc_shape(io_dtype=0)), 148, ctypes.byref(info)) == -5
     assert lib.kda_prefill_plan(ctypes.byref(tc_shape()), 148, None) == -1
     assert lib.kda_prefill_plan(None, 148, ctypes.byref(info)) == -1
+
+
+def test_python_binding_checks_shapes_before_the_device():
+    """Argument errors of the gated, layer and decode-layer calls are reported
+    as such (before the no-CPU-path check), so they surface on any machine."""
+    import torch
+    q = torch.zeros(1, 8, 2, 128)
+    beta = torch.zeros(1, 8, 2)
+    A, bias = torch.zeros(2), torch.zeros(2, 128)
+    with pytest.raises(ValueError, match="out_gate"):
+        kda.kda_chunk_fwd_gated(q, q, q, q, beta, torch.zeros(1, 8, 2, 64), torch.zeros(128))
+    with pytest.raises(ValueError, match="norm_weight"):
+        kda.kda_chunk_fwd_gated(q, q, q, q, beta, q, torch.zeros(64))
+    with pytest.raises(ValueError, match="gate_mode"):
+        kda.kda_chunk_fwd_gated(q, q, q, q, beta, q, torch.zeros(128), gate_mode="sometimes")
+    with pytest.raises(ValueError, match="gate_f"):
+        kda.kda_chunk_fwd_layer(q, q, q, torch.zeros(1, 8, 2, 64), A, bias, beta)
+    with pytest.raises(ValueError, match="A_log"):
+        kda.kda_chunk_fwd_layer(q, q, q, q, torch.zeros(3), bias, beta)
+    with pytest.raises(ValueError, match="go together"):
+        kda.kda_chunk_fwd_layer(q, q, q, q, A, bias, beta, out_gate=q)
+    with pytest.raises(ValueError, match="A_log"):
+        kda.kda_decode_step_layer(q[:, 0], q[:, 0], q[:, 0], q[:, 0], torch.zeros(5), bias, beta[:, 0],
+                                  torch.zeros(1, 2, 128, 128))
+    with pytest.raises(ValueError, match="CUDA"):
+        kda.kda_chunk_fwd_layer(q, q, q, q, A, bias, beta)
