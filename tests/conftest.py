@@ -11,6 +11,9 @@ if str(ROOT) not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
+    # temporary files of the tests (tmp_path) stay inside the repository
+    if not config.option.basetemp:
+        config.option.basetemp = str(ROOT / ".pytest_tmp")
 
 
 def pytest_collection_modifyitems(config, items):
